@@ -1,0 +1,120 @@
+"""Plant plausible mistakes in the oracle (CPU only) and check that the pins catch each one.
+
+A pin set that passes on a wrong oracle would not be evidence; every mutant below
+must make at least one test of ``test_oracle_pins`` fail.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import oracle.dsa_oracle as od
+import tests.test_oracle_pins as pins
+
+
+def _relu_after_sum(q, w, k):
+    return np.maximum(w @ (q @ k.T), 0.0)
+
+
+def _no_relu(q, w, k):
+    return w @ (q @ k.T)
+
+
+def _unweighted(q, w, k):
+    return np.maximum(q @ k.T, 0.0).sum(0)
+
+
+def _abs_weights(q, w, k):
+    return np.abs(w) @ np.maximum(q @ k.T, 0.0)
+
+
+def _ties_to_higher(scores, k):
+    n = scores.shape[0]
+    return np.lexsort((-np.arange(n), -scores))[: min(k, n)]
+
+
+def _bottom_k(scores, k):
+    n = scores.shape[0]
+    return np.lexsort((np.arange(n), scores))[: min(k, n)]
+
+
+def _value_is_rope_end(q, kv, d_v, tau):
+    out, lse = od.__dict__["_orig_attn"](q, kv, d_v, tau)
+    if kv.shape[0] == 0:
+        return out, lse
+    z = tau * (q @ kv.T)
+    p = np.exp(z - z.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    return p @ kv[:, -d_v:], lse
+
+
+def _lse_without_tau(q, kv, d_v, tau):
+    out, lse = od.__dict__["_orig_attn"](q, kv, d_v, tau)
+    if kv.shape[0] == 0:
+        return out, lse
+    z = q @ kv.T
+    return out, z.max(1) + np.log(np.exp(z - z.max(1, keepdims=True)).sum(1))
+
+
+def _softmax_over_heads(q, kv, d_v, tau):
+    if kv.shape[0] == 0:
+        return np.zeros((q.shape[0], d_v)), np.full(q.shape[0], -np.inf)
+    z = tau * (q @ kv.T)
+    p = np.exp(z - z.max(0, keepdims=True))
+    l = p.sum(0, keepdims=True)
+    return (p / l) @ kv[:, :d_v], z.max(1) + np.log(np.exp(z - z.max(1, keepdims=True)).sum(1))
+
+
+def _no_scale_e4m3(codes, scale=None):
+    return od._E4M3[np.asarray(codes, dtype=np.uint8)]
+
+
+def _e4m3_bias_8(codes, scale=None):
+    return od.__dict__["_orig_e4m3"](codes, scale) * 0.5
+
+
+MUTANTS = {
+    "relu_after_sum": ("index_scores", _relu_after_sum),
+    "no_relu": ("index_scores", _no_relu),
+    "unweighted_heads": ("index_scores", _unweighted),
+    "abs_weights": ("index_scores", _abs_weights),
+    "ties_to_higher": ("select_topk", _ties_to_higher),
+    "bottom_k": ("select_topk", _bottom_k),
+    "value_from_rope_end": ("sparse_mla_attention", _value_is_rope_end),
+    "lse_without_tau": ("sparse_mla_attention", _lse_without_tau),
+    "softmax_over_heads": ("sparse_mla_attention", _softmax_over_heads),
+    "scale_dropped": ("decode_e4m3", _no_scale_e4m3),
+    "e4m3_wrong_bias": ("decode_e4m3", _e4m3_bias_8),
+}
+
+PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
+
+
+def _run_pins():
+    failed = []
+    for fn in PIN_TESTS:
+        marks = getattr(fn, "pytestmark", [])
+        params = [m for m in marks if m.name == "parametrize"]
+        try:
+            if params:
+                names = [s.strip() for s in params[0].args[0].split(",")]
+                for vals in params[0].args[1]:
+                    fn(**dict(zip(names, vals)))
+            else:
+                fn()
+        except Exception:
+            failed.append(fn.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(mutant, monkeypatch):
+    name, fake = MUTANTS[mutant]
+    monkeypatch.setitem(od.__dict__, "_orig_attn", od.sparse_mla_attention)
+    monkeypatch.setitem(od.__dict__, "_orig_e4m3", od.decode_e4m3)
+    monkeypatch.setattr(od, name, fake)
+    monkeypatch.setattr(oracle, name, fake)
+    assert _run_pins(), f"no pin caught mutant {mutant}"
+
+
+def test_unmutated_oracle_passes_every_pin():
+    assert _run_pins() == []
