@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA forward path (lightning indexer + top-k + sparse MLA attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill_128k] [--impl ours|reference]
+
+One step = the whole hot path over one 128K-token causal prefill (B=1, L=131072, H_I=64,
+d_I=128 FP8, H=128, d_qk=576, d_v=512, k=2048), inputs resident in HBM, timed with CUDA
+events on the launching stream; metric = query-tokens/s. Under torchrun each rank runs its
+own independent sequence (weak scaling, no collective on the data path); timing is the max
+over ranks. Prints one JSON line on rank 0.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same workload (rank 0
+only; other ranks exit 0 without work).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synthetic  # noqa: E402
+
+METRIC = "DSA prefill query-tokens/s (indexer+top-k+sparse MLA) at 128K ctx, k=2048"
+UNIT = "query-tokens/s"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"], "bf16_sustained": d["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def _work(cfg):
+    """Algorithmic work per launch of each stage (causal prefill, B sequences of length L)."""
+    L, B = cfg.max_len, cfg.batch
+    pairs = B * L * (L + 1) // 2                              # causal (t, s) pairs, s <= t
+    k = min(cfg.topk, L)
+    sel_rows = B * (k * (k + 1) // 2 + (L - k) * cfg.topk)  # sum over t of min(k, t+1)
+    return {
+        "indexer_flop": pairs * 2 * cfg.n_idx_heads * cfg.idx_dim,                     # FP8 MACs x 2
+        "attn_flop": sel_rows * 2 * cfg.n_heads * (cfg.d_qk + cfg.d_v),                 # QK^T + PV
+        "attn_gather_bytes": sel_rows * cfg.d_qk * 2,
+        "pairs": pairs, "sel_rows": sel_rows,
+    }
+
+
+def _traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(path):
+        return None
+    import hashlib
+    src = os.path.join(ROOT, "sparse_attention_long_indexer_b200", "csrc",
+                       "indexer_topk.cuh" if kernel == "indexer" else "sparse_mla.cuh")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:12]
+    for line in open(path):
+        m = re.match(r"\|\s*(\w+)\s*\|\s*(\w+)\s*\|\s*([0-9.eE+]+)\s*\|\s*([0-9a-f]{12})\s*\|", line)
+        if m and m.group(1) == kernel and m.group(2) == workload and m.group(4) == sha:
+            return float(m.group(3))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms",
+                 "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [r for r in rows if r[2] > 300.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# ----------------------------------------------------------------------------- oracle timing (CPU)
+def _oracle_rows(cfg, seed, rows, cache=None):
+    """Runs the fp64 oracle (full path) on query rows of sequence 0.
+
+    Returns (oracle seconds, BLAS threads, cache); ``cache`` keeps the regenerated keys and
+    latent rows of the sequence so later calls only regenerate the per-query inputs."""
+    import oracle
+    from tests.dsa_cases import u16
+    if cache is None:
+        kc, ks = synthetic.gen_k_idx(cfg, seed, b=0)
+        cache = {"k": (kc.numpy(), ks.numpy()),
+                 "kv": u16(synthetic.gen_kv(cfg, seed, b=0, positions=range(0, cfg.max_len)))}
+    qc, qs = synthetic.gen_q_idx(cfg, seed, tokens=rows)
+    w = synthetic.gen_w(cfg, seed, tokens=rows)
+    q = synthetic.gen_q(cfg, seed, tokens=rows)
+    t0 = time.perf_counter()
+    for j, t in enumerate(rows):
+        oracle.dsa_row(qc[j].numpy(), float(qs[j]), u16(w[j]), cache["k"][0], cache["k"][1], u16(q[j]), cache["kv"],
+                       t, cfg.topk, cfg.d_v, cfg.softmax_scale)
+    dt = time.perf_counter() - t0
+    threads = 1
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        pass
+    return dt, threads, cache
+
+
+def _shuffled_rows(cfg, n, seed):
+    rows = synthetic.sample_rows(cfg.n_q, n, seed)
+    return [rows[i] for i in np.random.default_rng(seed).permutation(len(rows))]
+
+
+def cpu_baseline(cfg, seed, budget_s=20.0):
+    rows_all = _shuffled_rows(cfg, 4096, seed + 99)
+    t_start = time.perf_counter()
+    done, spent, cache, threads = 0, 0.0, None, 1
+    i = 0
+    while spent < budget_s and i < len(rows_all):
+        chunk = rows_all[i:i + 8]
+        dt, threads, cache = _oracle_rows(cfg, seed, chunk, cache)
+        spent += dt
+        done += len(chunk)
+        i += 8
+    return {"value": done / spent, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{done} seeded uniformly-random query rows of the {cfg.name} workload (full path per row: "
+                      f"fp64 index scores over keys 0..t, stable sort, fp64 attention over the k selected rows); "
+                      f"{spent:.1f} s of oracle time, {time.perf_counter() - t_start:.1f} s wall incl. input "
+                      f"regeneration"}
+
+
+# ----------------------------------------------------------------------------- multi-rank helpers
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own independent sequence (weak scaling)."""
+    return seed + rank
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank scalar over the process group (the job's time is its slowest rank)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(tokens_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: all ranks' query tokens over the slowest rank's time."""
+    return tokens_per_rank_step * steps * world / (max_ms / 1e3)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args, cfg, rank, world, local_rank):
+    import sparse_attention_long_indexer_b200 as dsa
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    seed = rank_seed(args.seed, rank)
+    g = synthetic.gen_all(cfg, seed, dev)
+    scales = torch.cat([g["q_scale"].reshape(-1), g["k_scale"].reshape(-1)]).contiguous()
+    dims = dsa.dims_for(cfg)
+    ws = dsa.Workspace.create(dims, cfg.topk, device=dev)
+    out = torch.empty((cfg.batch, cfg.n_q, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((cfg.batch, cfg.n_q, cfg.n_heads), dtype=torch.float32, device=dev)
+    idx = torch.empty((cfg.batch, cfg.n_q, cfg.topk), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dsa.dsa_indexer_topk(dims, g["q_idx"], g["w"], g["k_idx"], scales, g["lengths"], cfg.topk, idx, ws.buf, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        dsa.dsa_sparse_mla_attn(dims, g["q"], g["kv"], idx, cfg.topk, out, lse, ws.buf, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ws.check()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    end.record(stream)
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    ws.check()
+    total_ms = start.elapsed_time(end)
+    idx_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    att_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms = max_over_ranks(total_ms, dev)
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world)
+    return dict(total_ms=total_ms, idx_ms=idx_ms, att_ms=att_ms, clocks=clocks, e2e=e2e)
+
+
+def run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
+    """Same step, inputs copied from pinned host memory and results read back every step."""
+    names = ["q_idx", "w", "k_idx", "q", "kv", "lengths"]
+    try:
+        host = {k: torch.empty(g[k].shape, dtype=g[k].dtype, pin_memory=True) for k in names}
+        host_scales = torch.empty(scales.shape, dtype=scales.dtype, pin_memory=True)
+        host_out = torch.empty((cfg.batch, cfg.n_q, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, pin_memory=True)
+        host_lse = torch.empty((cfg.batch, cfg.n_q, cfg.n_heads), dtype=torch.float32, pin_memory=True)
+        host_idx = torch.empty((cfg.batch, cfg.n_q, cfg.topk), dtype=torch.int32, pin_memory=True)
+        pinned = True
+    except RuntimeError:
+        return {"value": None, "unit": UNIT, "note": "pinned host allocation failed"}
+    for k in names:
+        host[k].copy_(g[k])
+    host_scales.copy_(scales)
+    dev_in = {k: torch.empty_like(g[k]) for k in names}
+    dev_scales = torch.empty_like(scales)
+    out = torch.empty(host_out.shape, dtype=host_out.dtype, device=dev)
+    lse = torch.empty(host_lse.shape, dtype=host_lse.dtype, device=dev)
+    idx = torch.empty(host_idx.shape, dtype=host_idx.dtype, device=dev)
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names) + host_scales.numel() * 4
+    d2h = host_out.numel() * 2 + host_lse.numel() * 4 + host_idx.numel() * 4
+
+    def step():
+        for k in names:
+            dev_in[k].copy_(host[k], non_blocking=True)
+        dev_scales.copy_(host_scales, non_blocking=True)
+        dsa.dsa_forward(dims, dev_in["q_idx"], dev_in["w"], dev_in["k_idx"], dev_scales, dev_in["lengths"],
+                        cfg.topk, dev_in["q"], dev_in["kv"], idx, out, lse, ws.buf, stream)
+        host_out.copy_(out, non_blocking=True)
+        host_lse.copy_(lse, non_blocking=True)
+        host_idx.copy_(idx, non_blocking=True)
+
+    steps = max(1, min(args.steps, args.e2e_steps))
+    step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(a.elapsed_time(b), dev)
+    ws.check()
+    return {"value": aggregate_value(cfg.batch * cfg.n_q, steps, world, ms), "unit": UNIT, "steps": steps,
+            "ms_per_step": ms / steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pinned": pinned}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill_128k", choices=["prefill_4k", "prefill_32k", "prefill_128k"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    cfg = synthetic.config(args.workload)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return run_reference(args, cfg, world)
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    res = run_ours(args, cfg, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(report(args, cfg, res, world)), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def report(args, cfg, res, world):
+    peaks = _peaks()
+    w = _work(cfg)
+    ms_step = res["total_ms"] / args.steps
+    idx_ms = statistics.mean(res["idx_ms"])
+    att_ms = statistics.mean(res["att_ms"])
+    fp8_peak = 2.0 * peaks["bf16_sustained"]          # nominal fp8:bf16 ratio 2 (4.5 : 2.25 PF)
+    stages = {
+        "indexer_topk": {"ms": idx_ms, "bound": "tensor", "achieved": w["indexer_flop"] / (idx_ms / 1e3) / 1e12,
+                         "peak": fp8_peak, "unit": "TFLOP/s",
+                         "peak_note": f"fp8 = 2 x {peaks['source']} sustained bf16 {peaks['bf16_sustained']}"},
+        "sparse_mla_attn": {"ms": att_ms, "bound": "tensor", "achieved": w["attn_flop"] / (att_ms / 1e3) / 1e12,
+                            "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                            "peak_note": f"{peaks['source']} sustained bf16",
+                            "gather_GBps": w["attn_gather_bytes"] / (att_ms / 1e3) / 1e9},
+    }
+    for k, s in stages.items():
+        s["frac"] = s["achieved"] / s["peak"]
+    dom = "indexer_topk" if idx_ms >= att_ms else "sparse_mla_attn"
+    ds = stages[dom]
+    roofline = {"kernel": dom, "bound": ds["bound"], "achieved": ds["achieved"], "peak": ds["peak"],
+                "unit": ds["unit"], "frac": ds["frac"],
+                "traffic": _traffic("indexer" if dom == "indexer_topk" else "attention", cfg.name)}
+    line = {
+        "metric": METRIC, "value": aggregate_value(cfg.batch * cfg.n_q, args.steps, world, res["total_ms"]),
+        "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3+bf16 (fp32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: {cfg.description}; H_I={cfg.n_idx_heads} d_I={cfg.idx_dim} FP8 e4m3, "
+                               f"H={cfg.n_heads}, d_qk={cfg.d_qk}, d_v={cfg.d_v}, bf16",
+                   "global_batch": cfg.batch * world, "seq_len": cfg.max_len, "topk": cfg.topk,
+                   "parallelism": f"{world} independent sequences, one per GPU (no data-path collective)",
+                   "l2": "inputs larger than L2 (q alone is %.1f GB)" % (cfg.n_q * cfg.n_heads * cfg.d_qk * 2 / 1e9)},
+        "roofline": roofline, "stages": stages,
+        "gpu_launches": 2 * args.steps,
+        "clocks": res["clocks"], "e2e": res["e2e"],
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, args.seed, args.cpu_budget)
+    return line
+
+
+def run_reference(args, cfg, world):
+    """The fp64 oracle as the reference arm: each step is a bounded sample of the workload."""
+    rows_all = _shuffled_rows(cfg, 100000, args.seed + 7)
+    per_step = 4
+    cache = None
+    pos = 0
+    for _ in range(args.warmup):
+        _, _, cache = _oracle_rows(cfg, args.seed, rows_all[pos:pos + per_step], cache)
+        pos += per_step
+    total, threads = 0.0, 1
+    for _ in range(args.steps):
+        dt, threads, cache = _oracle_rows(cfg, args.seed, rows_all[pos:pos + per_step], cache)
+        total += dt
+        pos += per_step
+    value = per_step * args.steps / total
+    sample = (f"{per_step} seeded uniformly-random query rows per step of the {cfg.name} workload, full path per "
+              f"row (fp64 index scores, stable sort, fp64 attention)")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"{cfg.name}: {cfg.description}", "global_batch": cfg.batch,
+                       "seq_len": cfg.max_len, "topk": cfg.topk, "parallelism": "CPU oracle, rank 0 only"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,494 @@
+// Lightning indexer + fine-grained top-k selection, fused, for sm_100a.
+//
+// Computes, for every query t and every key s <= pos(t) of its sequence,
+//     I[t,s] = k_scale[s] * sum_j (w[t,j] * q_scale[t]) * ReLU(q8[t,j] . k8[s])
+// (the index score of the DeepSeek-V3.2-Exp summary "節前發版：Deepseek v3.2 exp",
+// section "Lightning indexer" Step 1, with the per-token FP8 scales of the inputs folded
+// out of the dot product: both are positive, so this equals sum_j w * ReLU(q . k) on the
+// decoded values), and keeps the k largest per query (Step 2), ties to the lower s.
+//
+// Design (one CTA per SM, persistent over work items):
+//  * a work item is NQ consecutive queries of one sequence and a contiguous key range;
+//  * TMA brings the item's query block [NQ*64 rows x 128 B] once and streams key tiles
+//    [128 keys x 128 B] through a ring of shared-memory stages (128-byte swizzle);
+//  * one thread issues tcgen05.mma kind::f8f6f4 (E4M3 x E4M3 -> f32), M = 128 keys,
+//    N = NQ*64 (query, head) columns, K = 128 in four steps, into one of two TMEM
+//    accumulators, so the MMA of tile i+1 overlaps the epilogue of tile i;
+//  * epilogue warps own one TMEM lane quarter each (a key per thread); they read the
+//    64 head columns of a query, apply ReLU and the weighted head sum in fp32 registers,
+//    mask s > pos(t), and append survivors of the per-query threshold into a candidate
+//    buffer in shared memory. When a buffer nears capacity, all epilogue warps run an exact
+//    radix select that keeps exactly k and raises the threshold. The L x L score matrix is
+//    never written anywhere.
+//  * prefill items cover a query block's whole causal key range and write the final
+//    indices; decode items (one query per sequence) cover a key chunk and write an exact
+//    partial top-k to the workspace, merged by `merge_partials_kernel`.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+#include "select.cuh"
+
+namespace dsa {
+
+constexpr int kIdxHeads = 64;     // H_I (padded)
+constexpr int kIdxDim = 128;      // d_I (padded), one 128-byte row per head / key
+constexpr int kKeyTile = 128;     // keys per MMA tile (M)
+constexpr int kCand = 3072;       // candidate capacity per query
+constexpr int kDecodeChunk = 8192;  // keys per decode work item
+
+template <int NQ>
+struct IdxCfg {
+  static constexpr int N = NQ * kIdxHeads;                 // MMA N
+  static constexpr int QPW = (NQ == 4) ? 2 : 1;            // queries per epilogue warp
+  static constexpr int EPI_WARPS = 4 * NQ / QPW;           // 8 or 4
+  static constexpr int EPI_THREADS = EPI_WARPS * 32;
+  static constexpr int PRODUCER_WARP = EPI_WARPS;
+  static constexpr int MMA_WARP = EPI_WARPS + 1;
+  static constexpr int THREADS = (EPI_WARPS + 2) * 32;
+  static constexpr int STAGES = (NQ == 4) ? 4 : 8;
+  static constexpr int Q_BYTES = NQ * kIdxHeads * kIdxDim;
+  static constexpr int K_BYTES = kKeyTile * kIdxDim;       // 16 KB
+  static constexpr int TMEM_COLS = 2 * N;                  // two accumulators
+  static constexpr int MAXPER = kCand / EPI_THREADS;
+  // shared-memory layout (offsets from a 1024-aligned base)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_KEYS = OFF_K + STAGES * K_BYTES;
+  static constexpr int OFF_POS = OFF_KEYS + NQ * kCand * 4;
+  static constexpr int OFF_W = OFF_POS + NQ * kCand * 4;
+  static constexpr int OFF_SEL = OFF_W + NQ * kIdxHeads * 4;
+  static constexpr int OFF_QST = OFF_SEL + static_cast<int>(sizeof(SelectScratch));
+  static constexpr int OFF_BAR = (OFF_QST + 3 * 4 * NQ + 8 + 16 + 7) & ~7;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 + 4 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static_assert(kCand % EPI_THREADS == 0, "candidate buffer must split evenly");
+  static_assert(Q_BYTES % 1024 == 0 && K_BYTES % 1024 == 0, "swizzle atoms");
+};
+
+struct IndexerParams {
+  const uint8_t* q_idx;     // [B, n_q, 64, 128] e4m3 (padded dims)
+  const __nv_bfloat16* w;   // [B, n_q, 64]
+  const float* q_scale;     // [B*n_q]
+  const float* k_scale;     // [B*max_len]
+  const int32_t* lengths;   // [B]
+  int32_t* out_idx;         // prefill: [B, n_q, topk]
+  uint32_t* part_keys;      // decode: [B, n_chunks, topk]
+  int32_t* part_pos;        // decode: [B, n_chunks, topk]
+  int32_t* part_count;      // decode: [B, n_chunks]
+  uint32_t* status;
+  int32_t batch, n_q, max_len, topk, n_chunks;
+  int32_t n_items;
+  uint64_t wait_budget_ns;
+};
+
+// Bounded wait that ignores the abort flag: used at teardown to let in-flight copies and
+// MMAs land before shared memory / TMEM are released. Gives up silently after the budget.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > budget_ns) return;
+  }
+}
+
+// Work item u -> (sequence, first query, key start, key end (exclusive), #tiles).
+struct Item {
+  int32_t b, i0, s_begin, s_end, ntiles, len;
+};
+
+template <int NQ>
+__device__ __forceinline__ Item make_item(const IndexerParams& p, int32_t u) {
+  Item it;
+  if (NQ == 1) {  // decode: key chunks of one query per sequence
+    it.b = u / p.n_chunks;
+    const int32_t c = u - it.b * p.n_chunks;
+    it.i0 = 0;
+    int32_t len = __ldg(p.lengths + it.b);
+    len = min(max(len, 0), p.max_len);
+    it.len = len;
+    const int32_t pos = len - p.n_q;          // the single query (i = 0)
+    it.s_begin = c * kDecodeChunk;
+    it.s_end = min(it.s_begin + kDecodeChunk, pos + 1);
+  } else {        // prefill: longest query blocks first
+    const int32_t nqb = (p.n_q + NQ - 1) / NQ;
+    const int32_t qb = nqb - 1 - u / p.batch;
+    it.b = u - (u / p.batch) * p.batch;
+    it.i0 = qb * NQ;
+    int32_t len = __ldg(p.lengths + it.b);
+    len = min(max(len, 0), p.max_len);
+    it.len = len;
+    const int32_t last_i = min(it.i0 + NQ, p.n_q) - 1;
+    const int32_t max_pos = len - p.n_q + last_i;
+    it.s_begin = 0;
+    it.s_end = max_pos + 1;
+  }
+  const int32_t span = it.s_end - it.s_begin;
+  it.ntiles = span > 0 ? (span + kKeyTile - 1) / kKeyTile : 0;
+  return it;
+}
+
+// Item sequence of CTA `cta` among `G`: snake order over rounds.
+__device__ __forceinline__ int32_t item_of(int32_t round, int32_t cta, int32_t G) {
+  return round * G + ((round & 1) ? (G - 1 - cta) : cta);
+}
+
+template <int NQ>
+__global__ void __launch_bounds__(IdxCfg<NQ>::THREADS, 1)
+indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                    const IndexerParams p) {
+  using C = IdxCfg<NQ>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint32_t* cand_keys = reinterpret_cast<uint32_t*>(smem + C::OFF_KEYS);
+  int32_t* cand_pos = reinterpret_cast<int32_t*>(smem + C::OFF_POS);
+  float* wq = reinterpret_cast<float*>(smem + C::OFF_W);
+  SelectScratch* sel = reinterpret_cast<SelectScratch*>(smem + C::OFF_SEL);
+  uint32_t* q_count = reinterpret_cast<uint32_t*>(smem + C::OFF_QST);
+  uint32_t* q_thr = q_count + NQ;
+  uint32_t* q_strict = q_thr + NQ;
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  auto k_full = [&](int s) { return bar0 + 8u * s; };
+  auto k_empty = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  const uint32_t q_full = bar0 + 8u * (2 * C::STAGES);
+  const uint32_t q_empty = q_full + 8;
+  auto acc_full = [&](int b) { return q_full + 16 + 8u * b; };
+  auto acc_empty = [&](int b) { return q_full + 32 + 8u * b; };
+  const uint32_t mma_done = q_full + 48;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full(b), 1);
+      mbar_init(acc_empty(b), C::EPI_WARPS);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  Waiter wt{p.status, abort_flag, p.wait_budget_ns, 1u};
+  const int32_t G = gridDim.x;
+  const int32_t cta = blockIdx.x;
+
+  if (warp == C::PRODUCER_WARP) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&map_q);
+      prefetch_tensormap(&map_k);
+      uint32_t stage = 0, phase = 0, qph = 0;
+      uint32_t used = 0, last_par = 0, q_out = 0;  // per stage: issued at least once / parity of last issue
+      for (int32_t r = 0;; ++r) {
+        const int32_t u = item_of(r, cta, G);
+        if (u >= p.n_items || wt.aborted()) break;
+        const Item it = make_item<NQ>(p, u);
+        if (it.ntiles == 0) continue;
+        if (!wt.wait(q_empty, qph ^ 1u, 1)) break;
+        q_out = 1u | (qph << 1);
+        qph ^= 1u;
+        mbar_expect_tx(q_full, C::Q_BYTES);
+        tma_load_3d(sbase + C::OFF_Q, &map_q, q_full, 0, it.i0 * kIdxHeads, it.b);
+        bool ok = true;
+        for (int32_t t = 0; t < it.ntiles; ++t) {
+          if (!wt.wait(k_empty(stage), phase ^ 1u, 2)) { ok = false; break; }
+          mbar_expect_tx(k_full(stage), C::K_BYTES);
+          tma_load_3d(sbase + C::OFF_K + stage * C::K_BYTES, &map_k, k_full(stage), 0,
+                      it.s_begin + t * kKeyTile, it.b);
+          used |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      // drain: every issued copy must have landed before the CTA may exit. Waiting on a
+      // completed phase returns at once; after an abort this bounds the in-flight copies.
+      for (int s = 0; s < C::STAGES; ++s)
+        if (used & (1u << s)) drain_wait(k_full(s), (last_par >> s) & 1u, p.wait_budget_ns);
+      if (q_out & 1u) drain_wait(q_full, (q_out >> 1) & 1u, p.wait_budget_ns);
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc(0, 0, 0, 0, kKeyTile, C::N);
+      uint32_t stage = 0, phase = 0, qph = 0, g = 0;
+      for (int32_t r = 0;; ++r) {
+        const int32_t u = item_of(r, cta, G);
+        if (u >= p.n_items || wt.aborted()) break;
+        const Item it = make_item<NQ>(p, u);
+        if (it.ntiles == 0) continue;
+        if (!wt.wait(q_full, qph, 4)) break;
+        qph ^= 1u;
+        bool ok = true;
+        for (int32_t t = 0; t < it.ntiles; ++t, ++g) {
+          const uint32_t buf = g & 1u, acc_ph = (g >> 1) & 1u;
+          if (!wt.wait(k_full(stage), phase, 5)) { ok = false; break; }
+          if (!wt.wait(acc_empty(buf), acc_ph ^ 1u, 6)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = sbase + C::OFF_K + stage * C::K_BYTES;
+          const uint32_t b_base = sbase + C::OFF_Q;
+#pragma unroll
+          for (int kk = 0; kk < kIdxDim / 32; ++kk) {
+            const uint64_t ad = sw128_desc(a_base + kk * 32, 1, 1024);
+            const uint64_t bd = sw128_desc(b_base + kk * 32, 1, 1024);
+            mma_f8_ss(tmem + buf * C::N, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(k_empty(stage));
+          tc_commit(acc_full(buf));
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        tc_commit(q_empty);
+        if (!ok) break;
+      }
+      // drain: all MMAs complete before TMEM is released
+      tc_commit(mma_done);
+      drain_wait(mma_done, 0, p.wait_budget_ns);
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue warps
+    // Named barriers (bar.sync) cannot time out, so every epilogue warp must take the same
+    // path through them: mbarrier waits are done by lane 0 and broadcast, and the decision
+    // to stop after an abort is a snapshot taken by one thread between two barriers.
+    const uint32_t etid = threadIdx.x;                   // 0 .. EPI_THREADS-1
+    const uint32_t quarter = warp & 3u;
+    const uint32_t qset = warp >> 2;                     // which QPW queries of the block
+    const uint32_t lane_base = (quarter * 32u) << 16;
+    volatile uint32_t* snap = q_strict + NQ;             // two parity slots
+    uint32_t g = 0, nsync = 0;
+    auto uniform_stop = [&]() -> bool {
+      named_barrier(1, C::EPI_THREADS);                  // every warp finished the step
+      if (etid == 0) snap[nsync & 1u] = (*abort_flag != 0) ? 1u : 0u;
+      named_barrier(1, C::EPI_THREADS);
+      return snap[(nsync++) & 1u] != 0;
+    };
+    bool stop = false;
+    for (int32_t r = 0; !stop; ++r) {
+      const int32_t u = item_of(r, cta, G);
+      if (u >= p.n_items) break;
+      const Item it = make_item<NQ>(p, u);
+      // per-query setup
+      for (uint32_t x = etid; x < NQ * kIdxHeads; x += C::EPI_THREADS) {
+        const int32_t i = it.i0 + static_cast<int32_t>(x / kIdxHeads);
+        float v = 0.f;
+        if (i < p.n_q) {
+          const size_t qt = static_cast<size_t>(it.b) * p.n_q + i;
+          v = __bfloat162float(p.w[qt * kIdxHeads + (x % kIdxHeads)]) * __ldg(p.q_scale + qt);
+        }
+        wq[x] = v;
+      }
+      if (etid < NQ) {
+        q_count[etid] = 0;
+        q_thr[etid] = 0;
+        q_strict[etid] = 0;
+      }
+      named_barrier(1, C::EPI_THREADS);
+      int32_t qpos[C::QPW];
+#pragma unroll
+      for (int j = 0; j < C::QPW; ++j) {
+        const int32_t i = it.i0 + static_cast<int32_t>(qset * C::QPW + j);
+        qpos[j] = (i < p.n_q) ? it.len - p.n_q + i : -1;
+      }
+      for (int32_t t = 0; t < it.ntiles; ++t, ++g) {
+        const uint32_t buf = g & 1u, acc_ph = (g >> 1) & 1u;
+        const int32_t s = it.s_begin + t * kKeyTile + static_cast<int32_t>(quarter * 32 + lane);
+        const bool in_range = s < it.s_end;
+        const float ks = in_range ? __ldg(p.k_scale + static_cast<size_t>(it.b) * p.max_len + s) : 0.f;
+        // lane 0 waits; the warp then runs the collective TMEM loads together
+        uint32_t got = 1;
+        if (lane == 0) got = wt.wait(acc_full(buf), acc_ph, 8) ? 1u : 0u;
+        const bool ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+        if (ok) {
+          uint32_t x[C::QPW][64];
+          tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < C::QPW; ++j) {
+            const uint32_t col = buf * C::N + (qset * C::QPW + j) * kIdxHeads;
+            tmem_ld32(tmem + lane_base + col, *reinterpret_cast<uint32_t(*)[32]>(&x[j][0]));
+            tmem_ld32(tmem + lane_base + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[j][32]));
+          }
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty(buf));
+#pragma unroll
+          for (int j = 0; j < C::QPW; ++j) {
+            const uint32_t q = qset * C::QPW + j;
+            const float4* w4 = reinterpret_cast<const float4*>(wq + q * kIdxHeads);
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+            for (int h = 0; h < kIdxHeads; h += 4) {
+              const float4 wv = w4[h / 4];
+              a0 = fmaf(wv.x, fmaxf(__uint_as_float(x[j][h + 0]), 0.f), a0);
+              a1 = fmaf(wv.y, fmaxf(__uint_as_float(x[j][h + 1]), 0.f), a1);
+              a2 = fmaf(wv.z, fmaxf(__uint_as_float(x[j][h + 2]), 0.f), a2);
+              a3 = fmaf(wv.w, fmaxf(__uint_as_float(x[j][h + 3]), 0.f), a3);
+            }
+            const float score = ((a0 + a1) + (a2 + a3)) * ks;
+            const uint32_t key = score_key(score);
+            const bool valid = in_range && s <= qpos[j];
+            const uint32_t thr = q_thr[q];
+            const bool pass = valid && (key > thr || (key == thr && q_strict[q] == 0));
+            const uint32_t m = __ballot_sync(0xffffffffu, pass);
+            if (m) {
+              uint32_t base = 0;
+              if (lane == 0) base = atomicAdd(&q_count[q], __popc(m));
+              base = __shfl_sync(0xffffffffu, base, 0);
+              if (pass) {
+                const uint32_t at = base + __popc(m & ((1u << lane) - 1u));
+                cand_keys[q * kCand + at] = key;
+                cand_pos[q * kCand + at] = s;
+              }
+            }
+          }
+        }
+        if (uniform_stop()) { stop = true; break; }
+        for (int q = 0; q < NQ; ++q) {
+          const uint32_t n = q_count[q];
+          if (n > static_cast<uint32_t>(kCand - kKeyTile)) {
+            const uint32_t vk = select_exact<C::EPI_THREADS, C::MAXPER>(
+                cand_keys + q * kCand, cand_pos + q * kCand, n, static_cast<uint32_t>(p.topk), sel, etid, 1);
+            if (etid == 0) {
+              q_count[q] = p.topk;
+              q_thr[q] = vk;
+              q_strict[q] = 1;
+            }
+            named_barrier(1, C::EPI_THREADS);
+          }
+        }
+      }
+      if (stop) break;
+      // ---- finish the item: exact k, then write
+      for (int q = 0; q < NQ; ++q) {
+        const int32_t i = it.i0 + q;
+        if (NQ > 1 && i >= p.n_q) break;
+        uint32_t n = q_count[q];
+        if (n > static_cast<uint32_t>(p.topk)) {
+          select_exact<C::EPI_THREADS, C::MAXPER>(cand_keys + q * kCand, cand_pos + q * kCand, n,
+                                                  static_cast<uint32_t>(p.topk), sel, etid, 1);
+          n = p.topk;
+        }
+        if (NQ == 1) {
+          const size_t slot = static_cast<size_t>(it.b) * p.n_chunks + (it.s_begin / kDecodeChunk);
+          for (uint32_t j = etid; j < n; j += C::EPI_THREADS) {
+            p.part_keys[slot * p.topk + j] = cand_keys[j];
+            p.part_pos[slot * p.topk + j] = cand_pos[j];
+          }
+          if (etid == 0) p.part_count[slot] = static_cast<int32_t>(n);
+        } else {
+          int32_t* dst = p.out_idx + (static_cast<size_t>(it.b) * p.n_q + i) * p.topk;
+          for (uint32_t j = etid; j < static_cast<uint32_t>(p.topk); j += C::EPI_THREADS)
+            dst[j] = j < n ? cand_pos[q * kCand + j] : -1;
+        }
+      }
+      named_barrier(1, C::EPI_THREADS);
+    }
+  }
+  // ---- teardown: every role reaches here (all waits are bounded)
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Decode: merge the per-chunk exact top-k lists of one sequence into its final top-k.
+// One CTA per sequence; candidates are read from the workspace (L2-resident).
+struct MergeParams {
+  const uint32_t* part_keys;
+  const int32_t* part_pos;
+  const int32_t* part_count;
+  int32_t* out_idx;        // [B, n_q(=1), topk]
+  int32_t n_chunks, topk;
+};
+
+template <int T>
+__global__ void __launch_bounds__(T) merge_partials_kernel(const MergeParams p) {
+  __shared__ SelectScratch sc;
+  __shared__ uint32_t s_count[1024 + 1];
+  const uint32_t tid = threadIdx.x;
+  const int32_t b = blockIdx.x;
+  const size_t base_slot = static_cast<size_t>(b) * p.n_chunks;
+  for (int32_t c = tid; c < p.n_chunks; c += T) s_count[c] = static_cast<uint32_t>(p.part_count[base_slot + c]);
+  __syncthreads();
+  uint32_t n = 0;
+  for (int32_t c = 0; c < p.n_chunks; ++c) n += s_count[c];
+  const uint32_t k = static_cast<uint32_t>(p.topk);
+  int32_t* dst = p.out_idx + static_cast<size_t>(b) * p.topk;
+  auto for_each = [&](auto&& fn) {
+    for (int32_t c = 0; c < p.n_chunks; ++c) {
+      const uint32_t* kk = p.part_keys + (base_slot + c) * p.topk;
+      const int32_t* pp = p.part_pos + (base_slot + c) * p.topk;
+      for (uint32_t j = tid; j < s_count[c]; j += T) fn(kk[j], pp[j]);
+    }
+  };
+  uint32_t vk = 0, plim = 0xFFFFFFFFu;
+  if (n > k) {
+    uint32_t prefix = 0, mask = 0, rem = k, n_eq = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (uint32_t i = tid; i < 256; i += T) sc.hist[i] = 0;
+      __syncthreads();
+      for_each([&](uint32_t key, int32_t) {
+        if ((key & mask) == prefix) atomicAdd(&sc.hist[(key >> shift) & 255u], 1u);
+      });
+      __syncthreads();
+      if (tid < 32) scan_pick<true>(&sc, rem);
+      __syncthreads();
+      rem -= sc.above;
+      n_eq = sc.hist[sc.bin];
+      prefix |= sc.bin << shift;
+      mask |= 0xFFu << shift;
+      __syncthreads();
+    }
+    vk = prefix;
+    if (rem < n_eq) {
+      uint32_t pprefix = 0, pmask = 0, prem = rem;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        for (uint32_t i = tid; i < 256; i += T) sc.hist[i] = 0;
+        __syncthreads();
+        for_each([&](uint32_t key, int32_t ps) {
+          const uint32_t pu = static_cast<uint32_t>(ps);
+          if (key == vk && (pu & pmask) == pprefix) atomicAdd(&sc.hist[(pu >> shift) & 255u], 1u);
+        });
+        __syncthreads();
+        if (tid < 32) scan_pick<false>(&sc, prem);
+        __syncthreads();
+        prem -= sc.above;
+        pprefix |= sc.bin << shift;
+        pmask |= 0xFFu << shift;
+        __syncthreads();
+      }
+      plim = pprefix;
+    }
+  }
+  if (tid == 0) sc.out_count = 0;
+  __syncthreads();
+  const bool all = n <= k;
+  for_each([&](uint32_t key, int32_t ps) {
+    if (all || key > vk || (key == vk && static_cast<uint32_t>(ps) <= plim)) {
+      const uint32_t at = atomicAdd(&sc.out_count, 1u);
+      if (at < k) dst[at] = ps;
+    }
+  });
+  __syncthreads();
+  for (uint32_t j = min(sc.out_count, k) + tid; j < k; j += T) dst[j] = -1;
+}
+
+}  // namespace dsa
