@@ -198,22 +198,38 @@ def run_ours(args, cfg, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     seed = rank_seed(args.seed, rank)
-    g = synthetic.gen_all(cfg, seed, dev)
-    scales = torch.cat([g["q_scale"].reshape(-1), g["k_scale"].reshape(-1)]).contiguous()
+    do_idx = args.stage in ("all", "indexer")
+    do_att = args.stage in ("all", "attention")
+    q_idx, q_scale = synthetic.gen_q_idx(cfg, seed, dev)
+    k_idx, k_scale = synthetic.gen_k_idx(cfg, seed, dev)
+    g = {"q_idx": q_idx, "k_idx": k_idx, "w": synthetic.gen_w(cfg, seed, dev),
+         "lengths": synthetic.lengths(cfg, seed).to(dev)}
+    if do_att:
+        g["q"] = synthetic.gen_q(cfg, seed, dev)
+        g["kv"] = synthetic.gen_kv(cfg, seed, dev)
+    scales = torch.cat([q_scale.reshape(-1), k_scale.reshape(-1)]).contiguous()
     dims = dsa.dims_for(cfg)
     ws = dsa.Workspace.create(dims, cfg.topk, device=dev)
-    out = torch.empty((cfg.batch, cfg.n_q, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((cfg.batch, cfg.n_q, cfg.n_heads), dtype=torch.float32, device=dev)
     idx = torch.empty((cfg.batch, cfg.n_q, cfg.topk), dtype=torch.int32, device=dev)
+    if do_att:
+        out = torch.empty((cfg.batch, cfg.n_q, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((cfg.batch, cfg.n_q, cfg.n_heads), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+
+    if not do_idx:   # the attention still needs real selections: compute them once, untimed
+        dsa.dsa_indexer_topk(dims, g["q_idx"], g["w"], g["k_idx"], scales, g["lengths"], cfg.topk, idx, ws.buf,
+                             stream)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        dsa.dsa_indexer_topk(dims, g["q_idx"], g["w"], g["k_idx"], scales, g["lengths"], cfg.topk, idx, ws.buf, stream)
+        if do_idx:
+            dsa.dsa_indexer_topk(dims, g["q_idx"], g["w"], g["k_idx"], scales, g["lengths"], cfg.topk, idx, ws.buf,
+                                 stream)
         if ev is not None:
             ev[1].record(stream)
-        dsa.dsa_sparse_mla_attn(dims, g["q"], g["kv"], idx, cfg.topk, out, lse, ws.buf, stream)
+        if do_att:
+            dsa.dsa_sparse_mla_attn(dims, g["q"], g["kv"], idx, cfg.topk, out, lse, ws.buf, stream)
         if ev is not None:
             ev[2].record(stream)
 
@@ -249,6 +265,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     if not args.no_e2e:
         e2e = run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world)
     return dict(total_ms=total_ms, idx_ms=idx_ms, att_ms=att_ms, clocks=clocks, e2e=e2e)
+
+
 
 
 def run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
@@ -314,10 +332,20 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--stage", default="all", choices=["all", "indexer", "attention"],
+                    help="time one stage only (profiling); the line then reports that stage")
+    ap.add_argument("--seq-len", type=int, default=0, help="override L of a prefill workload (profiling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     cfg = synthetic.config(args.workload)
+    if args.seq_len:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, n_q=args.seq_len, max_len=args.seq_len, name=f"prefill_L{args.seq_len}",
+                                  description=f"causal prefill L={args.seq_len}, k=2048")
+    if args.stage != "all":
+        args.no_e2e = True
+        args.no_cpu_baseline = True
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -348,18 +376,21 @@ def report(args, cfg, res, world):
     idx_ms = statistics.mean(res["idx_ms"])
     att_ms = statistics.mean(res["att_ms"])
     fp8_peak = 2.0 * peaks["bf16_sustained"]          # nominal fp8:bf16 ratio 2 (4.5 : 2.25 PF)
-    stages = {
-        "indexer_topk": {"ms": idx_ms, "bound": "tensor", "achieved": w["indexer_flop"] / (idx_ms / 1e3) / 1e12,
-                         "peak": fp8_peak, "unit": "TFLOP/s",
-                         "peak_note": f"fp8 = 2 x {peaks['source']} sustained bf16 {peaks['bf16_sustained']}"},
-        "sparse_mla_attn": {"ms": att_ms, "bound": "tensor", "achieved": w["attn_flop"] / (att_ms / 1e3) / 1e12,
-                            "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                            "peak_note": f"{peaks['source']} sustained bf16",
-                            "gather_GBps": w["attn_gather_bytes"] / (att_ms / 1e3) / 1e9},
-    }
+    stages = {}
+    if args.stage in ("all", "indexer"):
+        stages["indexer_topk"] = {"ms": idx_ms, "bound": "tensor",
+                                  "achieved": w["indexer_flop"] / (idx_ms / 1e3) / 1e12, "peak": fp8_peak,
+                                  "unit": "TFLOP/s",
+                                  "peak_note": f"fp8 = 2 x {peaks['source']} sustained bf16 {peaks['bf16_sustained']}"}
+    if args.stage in ("all", "attention"):
+        stages["sparse_mla_attn"] = {"ms": att_ms, "bound": "tensor",
+                                     "achieved": w["attn_flop"] / (att_ms / 1e3) / 1e12,
+                                     "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                                     "peak_note": f"{peaks['source']} sustained bf16",
+                                     "gather_GBps": w["attn_gather_bytes"] / (att_ms / 1e3) / 1e9}
     for k, s in stages.items():
         s["frac"] = s["achieved"] / s["peak"]
-    dom = "indexer_topk" if idx_ms >= att_ms else "sparse_mla_attn"
+    dom = max(stages, key=lambda k: stages[k]["ms"])
     ds = stages[dom]
     roofline = {"kernel": dom, "bound": ds["bound"], "achieved": ds["achieved"], "peak": ds["peak"],
                 "unit": ds["unit"], "frac": ds["frac"],
@@ -376,7 +407,7 @@ def report(args, cfg, res, world):
                    "parallelism": f"{world} independent sequences, one per GPU (no data-path collective)",
                    "l2": "inputs larger than L2 (q alone is %.1f GB)" % (cfg.n_q * cfg.n_heads * cfg.d_qk * 2 / 1e9)},
         "roofline": roofline, "stages": stages,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": len(stages) * args.steps,
         "clocks": res["clocks"], "e2e": res["e2e"],
     }
     if world == 1 and not args.no_cpu_baseline:

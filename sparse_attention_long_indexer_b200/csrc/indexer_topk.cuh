@@ -271,8 +271,11 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     const uint32_t lane_base = (quarter * 32u) << 16;
     volatile uint32_t* snap = q_strict + NQ;             // two parity slots
     uint32_t g = 0, nsync = 0;
+    // One barrier per step: thread 0 publishes the abort flag as it sees it into a parity
+    // slot before the barrier and everyone reads that slot after it. An abort raised while
+    // the slot was written is seen one step later, by all warps alike. A slot is rewritten
+    // two steps later, after every thread has read it.
     auto uniform_stop = [&]() -> bool {
-      named_barrier(1, C::EPI_THREADS);                  // every warp finished the step
       if (etid == 0) snap[nsync & 1u] = (*abort_flag != 0) ? 1u : 0u;
       named_barrier(1, C::EPI_THREADS);
       return snap[(nsync++) & 1u] != 0;
@@ -361,12 +364,22 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         for (int q = 0; q < NQ; ++q) {
           const uint32_t n = q_count[q];
           if (n > static_cast<uint32_t>(kCand - kKeyTile)) {
-            const uint32_t vk = select_exact<C::EPI_THREADS, C::MAXPER>(
-                cand_keys + q * kCand, cand_pos + q * kCand, n, static_cast<uint32_t>(p.topk), sel, etid, 1);
-            if (etid == 0) {
-              q_count[q] = p.topk;
-              q_thr[q] = vk;
-              q_strict[q] = 1;
+            // cheap range-histogram shrink; the exact select only if it frees too little
+            uint32_t thr = 0;
+            const uint32_t m = shrink_candidates<C::EPI_THREADS, C::MAXPER>(
+                cand_keys + q * kCand, cand_pos + q * kCand, n, static_cast<uint32_t>(p.topk), sel, etid, 1, &thr);
+            if (m > static_cast<uint32_t>((kCand + p.topk) / 2)) {
+              const uint32_t vk = select_exact<C::EPI_THREADS, C::MAXPER>(
+                  cand_keys + q * kCand, cand_pos + q * kCand, m, static_cast<uint32_t>(p.topk), sel, etid, 1);
+              if (etid == 0) {
+                q_count[q] = p.topk;
+                q_thr[q] = vk;
+                q_strict[q] = 1;
+              }
+            } else if (etid == 0) {
+              q_count[q] = m;
+              q_thr[q] = thr;
+              q_strict[q] = 0;
             }
             named_barrier(1, C::EPI_THREADS);
           }

@@ -27,6 +27,15 @@ struct SelectScratch {
   uint32_t pad;
 };
 
+// Adds 1 to hist[bin] for every lane with `active`, one shared atomic per distinct bin in
+// the warp (candidates cluster in few bins, so per-lane atomics would serialise).
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
+  const uint32_t lane = threadIdx.x & 31;
+  const uint32_t key = active ? bin : 0xFFFFFFFFu;
+  const uint32_t peers = __match_any_sync(0xffffffffu, key);
+  if (active && lane == static_cast<uint32_t>(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
+}
+
 // Warp 0 scans hist (bins descending when kDescending, else ascending) and publishes the bin
 // where the running count first reaches `rem`, with the count before it.
 template <bool kDescending>
@@ -70,9 +79,10 @@ __device__ uint32_t select_exact(uint32_t* keys, int32_t* pos, uint32_t n, uint3
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (uint32_t i = tid; i < 256; i += T) sc->hist[i] = 0;
     named_barrier(bar_id, T);
-    for (uint32_t i = tid; i < n; i += T) {
-      uint32_t key = keys[i];
-      if ((key & mask) == prefix) atomicAdd(&sc->hist[(key >> shift) & 255u], 1u);
+    for (uint32_t i0 = 0; i0 < n; i0 += T) {      // uniform trip count: hist_add is warp-collective
+      const uint32_t i = i0 + tid;
+      const uint32_t key = i < n ? keys[i] : 0u;
+      hist_add(sc->hist, (key >> shift) & 255u, i < n && (key & mask) == prefix);
     }
     named_barrier(bar_id, T);
     if (tid < 32) scan_pick<true>(sc, rem);
@@ -92,9 +102,10 @@ __device__ uint32_t select_exact(uint32_t* keys, int32_t* pos, uint32_t n, uint3
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (uint32_t i = tid; i < 256; i += T) sc->hist[i] = 0;
       named_barrier(bar_id, T);
-      for (uint32_t i = tid; i < n; i += T) {
-        uint32_t p = static_cast<uint32_t>(pos[i]);
-        if (keys[i] == vk && (p & pmask) == pprefix) atomicAdd(&sc->hist[(p >> shift) & 255u], 1u);
+      for (uint32_t i0 = 0; i0 < n; i0 += T) {
+        const uint32_t i = i0 + tid;
+        const uint32_t p = i < n ? static_cast<uint32_t>(pos[i]) : 0u;
+        hist_add(sc->hist, (p >> shift) & 255u, i < n && keys[i] == vk && (p & pmask) == pprefix);
       }
       named_barrier(bar_id, T);
       if (tid < 32) scan_pick<false>(sc, prem);
@@ -141,6 +152,80 @@ __device__ uint32_t select_exact(uint32_t* keys, int32_t* pos, uint32_t n, uint3
   }
   named_barrier(bar_id, T);
   return vk;
+}
+
+// Cheap shrink used while streaming: keeps every candidate whose key is at least the lower
+// edge of the histogram bin holding the k-th largest key, bins splitting the current key
+// range [min, max] into 256 equal intervals. At least k candidates stay (typically k plus a
+// few), and everything dropped is strictly below k kept ones, so the returned threshold is
+// non-strict: later candidates equal to it must still be admitted. Returns the new count;
+// `*thr_out` receives the threshold.
+template <int T, int MAXPER>
+__device__ uint32_t shrink_candidates(uint32_t* keys, int32_t* pos, uint32_t n, uint32_t k, SelectScratch* sc,
+                                      uint32_t tid, uint32_t bar_id, uint32_t* thr_out) {
+  const uint32_t lane = threadIdx.x & 31;
+  uint32_t rk[MAXPER];
+  int32_t rp[MAXPER];
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+  for (int j = 0; j < MAXPER; ++j) {
+    const uint32_t i = tid + j * T;
+    rk[j] = 0;
+    rp[j] = -1;
+    if (i < n) {
+      rk[j] = keys[i];
+      rp[j] = pos[i];
+      lo = min(lo, rk[j]);
+      hi = max(hi, rk[j]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  for (uint32_t i = tid; i < 256; i += T) sc->hist[i] = 0;
+  if (tid == 0) {
+    sc->bin = 0xFFFFFFFFu;   // running min
+    sc->above = 0u;          // running max
+  }
+  named_barrier(bar_id, T);
+  if (lane == 0) {
+    atomicMin(&sc->bin, lo);
+    atomicMax(&sc->above, hi);
+  }
+  named_barrier(bar_id, T);
+  lo = sc->bin;
+  hi = sc->above;
+  const uint32_t range = hi - lo;
+  const uint32_t shift = range < 256u ? 0u : (32u - __clz(range)) - 8u;
+#pragma unroll
+  for (int j = 0; j < MAXPER; ++j) hist_add(sc->hist, (rk[j] - lo) >> shift, rp[j] >= 0);
+  named_barrier(bar_id, T);
+  if (tid < 32) scan_pick<true>(sc, k);
+  named_barrier(bar_id, T);
+  const uint32_t thr = lo + (sc->bin << shift);
+  if (tid == 0) sc->out_count = 0;
+  named_barrier(bar_id, T);
+#pragma unroll
+  for (int j = 0; j < MAXPER; ++j) {
+    const bool keep = rp[j] >= 0 && rk[j] >= thr;
+    const uint32_t m = __ballot_sync(0xffffffffu, keep);
+    if (m) {
+      uint32_t base = 0;
+      const uint32_t leader = __ffs(m) - 1;
+      if (lane == leader) base = atomicAdd(&sc->out_count, __popc(m));
+      base = __shfl_sync(0xffffffffu, base, leader);
+      if (keep) {
+        const uint32_t at = base + __popc(m & ((1u << lane) - 1u));
+        keys[at] = rk[j];
+        pos[at] = rp[j];
+      }
+    }
+  }
+  named_barrier(bar_id, T);
+  *thr_out = thr;
+  return sc->out_count;
 }
 
 }  // namespace dsa

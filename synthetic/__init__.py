@@ -18,8 +18,8 @@ Determinism across devices.  Every element is a pure function of
   approximation of a normal law with mean 0 and unit variance after scaling);
   the sum is an exact integer below 2**18, converted exactly to fp32 and
   multiplied once by an fp32 constant (one IEEE-rounded product);
-* FP8 quantisation divides by the per-token scale amax/448 (one IEEE-rounded
-  quotient), clamps to the E4M3 range and rounds to nearest-even; bf16 is a
+* FP8 quantisation uses a per-token power-of-two scale (exact scaling, below
+  the E4M3 maximum) and one round-to-nearest-even cast; bf16 is a
   round-to-nearest-even cast.
 
 So a row generated on the CPU for the oracle has the same bits as the same row
@@ -189,11 +189,25 @@ def normal_rows(seed: int, tensor: str, rows, row_len: int, std: float, device="
     return _irwin_hall(rid[:, None] * row_len + cols[None, :], key, std)
 
 
+def _pow2(k: torch.Tensor) -> torch.Tensor:
+    """2**k in fp32 built from its IEEE bits (exact; k clamped to the normal range)."""
+    return ((k.to(torch.int32) + 127).clamp(1, 254) << 23).view(torch.float32)
+
+
 def quantize_e4m3_rows(x: torch.Tensor):
-    """Per-row FP8 E4M3 codes (uint8) and fp32 scales, scale = amax/448 (1 if amax == 0)."""
+    """Per-row FP8 E4M3 codes (uint8) and fp32 scales.
+
+    The scale is the power of two 2**(e-8) where amax = m * 2**e, 0.5 <= m < 1 (1 if
+    amax == 0), so |x / scale| < 256 <= 448 and x / scale is exact; the only rounding is
+    the round-to-nearest-even cast to E4M3. (A division by amax/448 would round twice, and
+    torch rounds a division by a Python scalar differently on CPU and CUDA.)
+    """
     amax = x.abs().amax(dim=1)
-    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
-    y = torch.clamp(x / scale[:, None], -E4M3_MAX, E4M3_MAX)
+    _, e = torch.frexp(amax)
+    nz = amax > 0
+    scale = torch.where(nz, _pow2(e - 8), torch.ones_like(amax))
+    inv = torch.where(nz, _pow2(8 - e), torch.zeros_like(amax))
+    y = x * inv[:, None]
     return y.to(torch.float8_e4m3fn).view(torch.uint8), scale
 
 

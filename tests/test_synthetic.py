@@ -42,16 +42,25 @@ def test_moments_are_standard_normal_like():
     assert x.abs().max().item() <= 2.0 * math.sqrt(12.0) + 1e-5      # Irwin-Hall(4) bound
 
 
-def test_e4m3_quantisation_uses_amax_over_448():
+def test_e4m3_quantisation_uses_exact_power_of_two_scales():
     x = synthetic.normal_rows(3, "q_idx", range(0, 64), 256, 1.0)
+    x[5] = 0.0
     codes, scale = synthetic.quantize_e4m3_rows(x)
+    s = scale.double().numpy()
+    m, _ = np.frexp(s)
+    assert (m == 0.5).all()                                    # powers of two
     dec = oracle.decode_e4m3(codes.numpy(), scale.numpy())
-    amax = x.abs().amax(1).double().numpy()
-    assert np.allclose(scale.double().numpy(), amax / 448.0, rtol=1e-6)
-    assert np.allclose(np.abs(dec).max(1), amax, rtol=1e-6)
-    err = np.abs(dec - x.double().numpy())
-    assert (err <= np.maximum(np.abs(x.double().numpy()) * 2.0 ** -4, scale.double().numpy()[:, None] * 2 ** -9)
-            + 1e-12).all()
+    xd = x.double().numpy()
+    amax = np.abs(xd).max(1)
+    nz = amax > 0
+    assert (amax[nz] / s[nz] < 256).all() and (amax[nz] / s[nz] >= 128).all()
+    assert (dec[~nz] == 0).all() and (s[~nz] == 1).all()
+    # round to nearest: within half an E4M3 step of the exact scaled value
+    err = np.abs(dec - xd)
+    assert (err <= np.maximum(np.abs(xd) * 2.0 ** -4, s[:, None] * 2.0 ** -10) + 1e-30).all()
+    # and exactly the RNE cast of x / scale
+    ref = torch.from_numpy(xd / s[:, None]).float().to(torch.float8_e4m3fn).view(torch.uint8)
+    assert torch.equal(ref, codes)
 
 
 def test_row_subsets_match_full_generation():
