@@ -332,17 +332,24 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
 #pragma unroll
           for (int j = 0; j < C::QPW; ++j) {
             const uint32_t q = qset * C::QPW + j;
+            // sum_j w'_j * ReLU(x_j): packed fp32x2 FMAs over 4 independent accumulator pairs
             const float4* w4 = reinterpret_cast<const float4*>(wq + q * kIdxHeads);
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
 #pragma unroll
             for (int h = 0; h < kIdxHeads; h += 4) {
               const float4 wv = w4[h / 4];
-              a0 = fmaf(wv.x, fmaxf(__uint_as_float(x[j][h + 0]), 0.f), a0);
-              a1 = fmaf(wv.y, fmaxf(__uint_as_float(x[j][h + 1]), 0.f), a1);
-              a2 = fmaf(wv.z, fmaxf(__uint_as_float(x[j][h + 2]), 0.f), a2);
-              a3 = fmaf(wv.w, fmaxf(__uint_as_float(x[j][h + 3]), 0.f), a3);
+              const float2 r01 = make_float2(fmaxf(__uint_as_float(x[j][h + 0]), 0.f),
+                                             fmaxf(__uint_as_float(x[j][h + 1]), 0.f));
+              const float2 r23 = make_float2(fmaxf(__uint_as_float(x[j][h + 2]), 0.f),
+                                             fmaxf(__uint_as_float(x[j][h + 3]), 0.f));
+              const int c = (h / 4) & 1;
+              acc[2 * c] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc[2 * c]);
+              acc[2 * c + 1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc[2 * c + 1]);
             }
-            const float score = ((a0 + a1) + (a2 + a3)) * ks;
+            const float score =
+                (((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y))) *
+                ks;
             const uint32_t key = score_key(score);
             const bool valid = in_range && s <= qpos[j];
             const uint32_t thr = q_thr[q];
