@@ -118,6 +118,30 @@ dsa_status dsa_forward(const dsa_dims* dims, const void* q_idx, const void* w, c
                        const void* latent_kv, int32_t* out_idx, void* out, float* lse, void* ws,
                        size_t ws_bytes, dsa_stream_t stream);
 
+/*
+ * Decode selection without a workspace, for callers that cannot allocate device memory
+ * for a call (serving runtimes that plan every buffer ahead and forbid allocation on the
+ * request path, plugin interfaces that pass a kernel only its inputs and outputs, loops
+ * where cudaMalloc's implicit synchronisation is not acceptable). The pages have no
+ * counterpart: this is a deployment variant of dsa_indexer_topk for n_q = 1.
+ *
+ * Same inputs, output and selection rule as dsa_indexer_topk with n_q = 1 and the
+ * production dims (64 indexer heads of dim 128). Its scratch -- the exact top-k list of
+ * every (sequence, 8192-key chunk) pair before the merge -- lives in a file-scope device
+ * array of the library (16 MiB + 4 KiB, held by every GPU that loads the library until the
+ * process exits), so the call allocates nothing and needs no workspace.
+ *   status  optional device pointer to 2 uint32 words: a device-side error (see dsa_status)
+ *           is recorded there, first error wins; the caller zeroes and reads it. May be NULL.
+ * Limits: batch * ceil(max_len / 8192) <= 1024 and topk <= 2048, else DSA_ERR_UNSUPPORTED
+ * (also for n_q != 1 or other dims). The first call on a device looks up the array's device
+ * address; make that first call before any stream capture. All calls on one device share
+ * the one array: two calls whose executions overlap on the GPU (for example on different
+ * streams) race and corrupt each other's results.
+ */
+dsa_status dsa_indexer_topk_decode_noalloc(const dsa_dims* dims, const void* q_idx, const void* w,
+                                           const void* k_idx, const float* scales, const int32_t* lengths,
+                                           int32_t topk, int32_t* out_idx, uint32_t* status, dsa_stream_t stream);
+
 /* Synchronises `stream`, returns the first device-side error recorded in `ws` since the
  * last call (DSA_OK if none) and clears it. `detail`, if non-NULL, receives a location tag. */
 dsa_status dsa_get_device_status(void* ws, dsa_stream_t stream, uint32_t* detail);

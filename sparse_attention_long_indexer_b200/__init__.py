@@ -30,7 +30,8 @@ DSA_ERR_DEVICE_TIMEOUT, DSA_ERR_INDEX_RANGE, DSA_ERR_WORKSPACE = 4, 5, 6
 
 LIBRARY_PATH = _LIB_PATH
 EXPORTED = ("dsa_workspace_bytes", "dsa_workspace_init", "dsa_indexer_topk", "dsa_sparse_mla_attn",
-            "dsa_forward", "dsa_get_device_status", "dsa_status_string", "dsa_version")
+            "dsa_forward", "dsa_get_device_status", "dsa_status_string", "dsa_version",
+            "dsa_indexer_topk_decode_noalloc")
 
 
 class dsa_dims(ctypes.Structure):

@@ -457,3 +457,92 @@ const char* dsa_status_string(dsa_status status) {
 int32_t dsa_version(void) { return 100; }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------- decode without a workspace
+// Some callers cannot allocate device memory for a call: serving runtimes that plan every
+// buffer ahead and forbid allocation on the request path, plugin interfaces that hand a kernel
+// only its inputs and outputs, and latency-critical loops where cudaMalloc's implicit device
+// synchronisation is unacceptable. For them, the decode selection (one query per sequence)
+// has a variant whose scratch -- the exact per-chunk top-k lists merged into the final
+// selection -- lives in this file-scope device array instead of a caller workspace. The array
+// is sized for kStaticSlots (sequence, 8192-key chunk) pairs at top-k <= 2048 (16 MiB plus the
+// counts); every GPU that loads the library keeps it until the process exits.
+namespace {
+
+constexpr size_t kStaticSlots = 1024;
+constexpr size_t kStaticTopk = 2048;
+constexpr size_t kStaticKeysBytes = kStaticSlots * kStaticTopk * 4;
+constexpr size_t kStaticBytes = 2 * kStaticKeysBytes + kStaticSlots * 4;
+
+static __device__ __align__(256) uint8_t g_decode_scratch[kStaticBytes];
+
+// Device address of g_decode_scratch on the current device, looked up once per device.
+dsa_status static_scratch(uint8_t** out) {
+  static std::mutex mu;
+  static uint8_t* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> g(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return DSA_ERR_CUDA;
+    addr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = addr[dev];
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" dsa_status dsa_indexer_topk_decode_noalloc(const dsa_dims* dims, const void* q_idx, const void* w,
+                                                      const void* k_idx, const float* scales, const int32_t* lengths,
+                                                      int32_t topk, int32_t* out_idx, uint32_t* status,
+                                                      dsa_stream_t stream) {
+  dsa_status s = check_dims(dims, topk);
+  if (s != DSA_OK) return s;
+  const dsa_dims& d = *dims;
+  if (d.n_q != 1 || !is_production(d)) return DSA_ERR_UNSUPPORTED;
+  const int32_t n_chunks = (d.max_len + kDecodeChunk - 1) / kDecodeChunk;
+  if (static_cast<size_t>(d.batch) * n_chunks > kStaticSlots || static_cast<size_t>(topk) > kStaticTopk)
+    return DSA_ERR_UNSUPPORTED;
+  if (d.batch == 0) return DSA_OK;
+  if (!q_idx || !w || !k_idx || !scales || !lengths || !out_idx) return DSA_ERR_INVALID_ARG;
+  if (!aligned(q_idx, 16) || !aligned(k_idx, 16) || !aligned(w, 2) || !aligned(scales, 4) ||
+      !aligned(lengths, 4) || !aligned(out_idx, 4) || (status != nullptr && !aligned(status, 4)))
+    return DSA_ERR_INVALID_ARG;
+  if ((s = device_ok()) != DSA_OK) return s;
+  uint8_t* scratch = nullptr;
+  if ((s = static_scratch(&scratch)) != DSA_OK) return s;
+  const DeviceInfo dev = device_info();
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  IndexerParams p{};
+  p.q_idx = static_cast<const uint8_t*>(q_idx);
+  p.w = static_cast<const __nv_bfloat16*>(w);
+  p.q_scale = scales;
+  p.k_scale = scales + d.batch;
+  p.lengths = lengths;
+  p.out_idx = out_idx;
+  p.status = status;
+  p.batch = d.batch;
+  p.n_q = 1;
+  p.max_len = d.max_len;
+  p.topk = topk;
+  p.wait_budget_ns = kWaitBudgetNs;
+  p.n_chunks = n_chunks;
+  // the slots are laid out with the call's top-k as row width; every slot a call reads is
+  // written earlier in the same call, so stale contents from a previous call are never used
+  p.part_keys = reinterpret_cast<uint32_t*>(scratch);
+  p.part_pos = reinterpret_cast<int32_t*>(scratch + kStaticKeysBytes);
+  p.part_count = reinterpret_cast<int32_t*>(scratch + 2 * kStaticKeysBytes);
+  p.n_items = d.batch * n_chunks;
+  CUtensorMap map_q, map_k;
+  if (!encode_rows_u8(&map_k, k_idx, static_cast<uint64_t>(d.max_len), static_cast<uint64_t>(d.batch), kKeyTile) ||
+      !encode_rows_u8(&map_q, q_idx, static_cast<uint64_t>(kIdxHeads), static_cast<uint64_t>(d.batch), kIdxHeads))
+    return DSA_ERR_CUDA;
+  const int grid = std::min(p.n_items, dev.sms);
+  indexer_topk_kernel<1><<<grid, IdxCfg<1>::THREADS, IdxCfg<1>::SMEM_BYTES, st>>>(map_q, map_k, p);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  MergeParams mp{p.part_keys, p.part_pos, p.part_count, out_idx, n_chunks, topk};
+  merge_partials_kernel<512><<<d.batch, 512, 0, st>>>(mp);
+  return from_cuda(cudaGetLastError());
+}
