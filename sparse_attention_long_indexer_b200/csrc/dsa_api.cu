@@ -189,6 +189,19 @@ bool encode_rows_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Queries as a 2-D bf16 tensor [rows = B*n_q*128 heads, 576 dims], box {64 dims, 64 heads}.
+bool encode_q_bf16(CUtensorMap* map, const void* base, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDqk), rows, 1};
+  const cuuint64_t strides[2] = {kDqk * 2, rows * kDqk * 2};
+  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 dsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
@@ -277,8 +290,10 @@ dsa_status run_attention(const dsa_dims& d, const __nv_bfloat16* q, const __nv_b
   p.n_queries = d.batch * d.n_q;
   p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
   p.wait_budget_ns = kWaitBudgetNs;
+  CUtensorMap map_q;
+  if (!encode_q_bf16(&map_q, q, static_cast<uint64_t>(p.n_queries) * kHeads)) return DSA_ERR_CUDA;
   const int clusters = std::max(1, std::min(p.n_queries, dev.sms / 2));
-  sparse_mla_attn_kernel<<<2 * clusters, AttnCfg::THREADS, AttnCfg::SMEM_BYTES, st>>>(p);
+  sparse_mla_attn_kernel<<<2 * clusters, AttnCfg::THREADS, AttnCfg::SMEM_BYTES, st>>>(map_q, p);
   return from_cuda(cudaGetLastError());
 }
 

@@ -7,20 +7,30 @@
 // "在MLA下實例化DSA": attention runs only over the selected entries, and in MLA's MQA mode
 // every query head shares the one latent vector of each token).
 //
-// B200 design. The fp32 output accumulator of one query, 128 heads x 512 dims, is 256 KB:
-// all of one SM's tensor memory. So each query runs on a cluster of two CTAs (two SMs):
-//  * CTA r keeps output columns [256r, 256r+256) in TMEM (256 columns) and the query's
-//    dims [288r, 288r+288) in TMEM (144 columns, the A operand of the QK^T MMA);
-//  * per block of 64 selected rows, CTA r gathers the dims it needs (r=0: [0,288), r=1:
-//    [256,576)) with 16-byte cp.async into a 128-byte-swizzled stage, and computes the
-//    partial logits S_r = Q[:,dims_r] . K[:,dims_r]^T on tcgen05 (kind::f16, A from TMEM);
-//  * the two fp32 partials are swapped through distributed shared memory and summed in a
-//    fixed order, so both CTAs hold bit-identical logits and take identical softmax steps;
-//  * P (bf16) goes to TMEM and O_r += P . V[:, 256r:256r+256] runs on tcgen05 with the same
-//    stage read as an MN-major operand; the softmax is online in the log2 domain, rescaling
-//    O only when the running max grows by more than 8 (exact: the final division uses the
-//    same stale max).
-// Each gathered row is thus shared by all 128 heads as a dense [128 x d] x [d x 64] product.
+// B200 design. The fp32 output accumulator of one query (128 heads x 512 dims) is 256 KB,
+// all of one SM's tensor memory, so each query runs on a pair of CTAs (a 2-CTA cluster) and
+// every product is a 2-SM tcgen05 MMA (cta_group::2) issued by one thread of the even CTA:
+//  * logits: M = 128 heads (CTA r supplies heads 64r..64r+63), N = 64 selected rows (CTA r
+//    supplies block rows 32r..32r+31), K = 576. The hardware shares the halves and each CTA
+//    receives the logits of its own 64 heads for all 64 rows, folded in TMEM as 128 lanes x
+//    32 columns (lane m: rows 0..31 of head m, lane 64+m: rows 32..63). Dims 0..287 of Q come
+//    from TMEM (A operand, duplicated over both lane halves), dims 288..575 from shared memory.
+//  * output: M = 128 heads, N = 256 latent dims per instruction (two instructions), K = 64
+//    rows: A = P (bf16, this CTA's heads) in shared memory, B = the rows' latent dims with CTA
+//    r supplying dims 256i + 128r .. +127. Each CTA accumulates all 512 dims of its 64 heads
+//    (TMEM: 256 columns; lane m / 64+m hold the low / high 128 dims of each instruction).
+//  * per 64-row block, CTA r gathers its 32 rows completely (logits operand, a 3-stage ring
+//    freed by the logits MMA) and all 64 rows' dims it supplies to the output product (a
+//    2-stage ring freed by the output MMA), with 16-byte cp.async into 128-byte-swizzled
+//    stages; two producer warp pairs run the two rings independently.
+//  * softmax: one thread per TMEM lane holds half a row (32 logits); the two halves of a row
+//    exchange their maxima through shared memory; online softmax in the log2 domain, the
+//    output rescaled only when the running max grows by more than 8 (exact: the final
+//    normalisation uses the same max). The logits of block b+1 are computed while the
+//    softmax of block b runs (two TMEM logit buffers).
+// Nothing crosses between the two CTAs except through the 2-SM MMAs themselves; the pair
+// synchronises through mbarriers of the even CTA (remote arrives) and commits that the MMA
+// thread addresses to both CTAs.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -36,28 +46,39 @@ constexpr int kBlk = 64;                 // selected rows per block
 constexpr int kMaxTopk = 2048;
 
 struct AttnCfg {
-  static constexpr int STAGES = 3;
-  static constexpr int ATOMS = 5;                        // 5 x 64 dims per stage row
-  static constexpr int ATOM_BYTES = kBlk * 128;          // 8 KB
-  static constexpr int STAGE_BYTES = ATOMS * ATOM_BYTES; // 40 KB
-  static constexpr int X_BYTES = kHeads * kBlk * 4;      // 32 KB partial logits
-  static constexpr int SOFTMAX_WARPS = 4;                // warp w owns TMEM lanes 32w..32w+31
-  static constexpr int PRODUCER_WARPS = 4;
-  static constexpr int PRODUCER_THREADS = PRODUCER_WARPS * 32;
+  static constexpr int SB_STAGES = 3;                    // own rows, all dims (logits operand)
+  static constexpr int VR_STAGES = 2;                    // all rows, this CTA's output dims
+  static constexpr int SB_ATOM = 32 * 128;               // 32 rows x 128 B
+  static constexpr int SB_BYTES = 9 * SB_ATOM;           // own 32 rows x 576 dims
+  static constexpr int VR_ATOM = kBlk * 128;             // 64 rows x 128 B
+  static constexpr int VR_BYTES = 4 * VR_ATOM;           // 64 rows x this CTA's 256 output dims
+  static constexpr int Q_TMEM_DIMS = 384;                // dims 0..383 of q in TMEM, the rest in smem
+  static constexpr int QS_ATOMS = (kDqk - Q_TMEM_DIMS) / 64;
+  static constexpr int QS_BYTES = QS_ATOMS * 64 * 128;   // 64 heads x dims 384..575
+  static constexpr int P_BYTES = 64 * 128;               // 64 heads x 64 rows bf16
+  static constexpr int SOFTMAX_WARPS = 4;
+  static constexpr int PRODUCER_WARPS = 4;               // 2 gather the logits ring, 2 the output ring
+  static constexpr int GROUP_THREADS = 64;
   static constexpr int MMA_WARP = SOFTMAX_WARPS + PRODUCER_WARPS;
   static constexpr int THREADS = (MMA_WARP + 1) * 32;
   // TMEM columns
-  static constexpr uint32_t COL_O = 0, COL_S = 256, COL_P = 320, COL_Q = 352, TMEM_COLS = 512;
+  static constexpr uint32_t COL_O = 0, COL_S = 256, COL_Q = 320, TMEM_COLS = 512;
   // shared memory
-  static constexpr int OFF_STAGE = 0;
-  static constexpr int OFF_X = OFF_STAGE + STAGES * STAGE_BYTES;
-  static constexpr int OFF_SEL = OFF_X + 2 * X_BYTES;
-  static constexpr int OFF_SCAN = OFF_SEL + kMaxTopk * 4;
-  static constexpr int OFF_INFO = OFF_SCAN + 64;   // scan: 4 warp sums + 2 go slots
+  static constexpr int OFF_SB = 0;
+  static constexpr int OFF_VR = OFF_SB + SB_STAGES * SB_BYTES;
+  static constexpr int OFF_QS = OFF_VR + VR_STAGES * VR_BYTES;
+  static constexpr int OFF_P = OFF_QS + QS_BYTES;
+  static constexpr int OFF_SEL = OFF_P + P_BYTES;                  // 2 x kMaxTopk indices
+  static constexpr int OFF_XMAX = OFF_SEL + 2 * kMaxTopk * 4;      // 2 x 128 floats
+  static constexpr int OFF_SCAN = OFF_XMAX + 2 * 128 * 4;
+  static constexpr int OFF_INFO = OFF_SCAN + 64;
   static constexpr int OFF_BAR = OFF_INFO + 16;
-  static constexpr int NUM_BARS = 2 * STAGES + 7 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int NUM_BARS = 40;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(OFF_VR % 1024 == 0 && OFF_QS % 1024 == 0 && OFF_P % 1024 == 0, "swizzle atoms");
+  static_assert(SB_BYTES % 1024 == 0 && Q_TMEM_DIMS / 2 + COL_Q <= TMEM_COLS, "layout");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 struct AttnParams {
@@ -85,225 +106,378 @@ __device__ __forceinline__ void attn_drain_wait(uint32_t bar, uint32_t parity, u
   }
 }
 
+// 2-SM MMAs (issued by one thread of the even CTA; operands at the same shared-memory
+// offsets / TMEM columns in both CTAs) and commits to an mbarrier of either CTA.
+__device__ __forceinline__ void mma2_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+               ::"r"(d), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+__device__ __forceinline__ void mma2_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+               ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+__device__ __forceinline__ void commit2(uint32_t bar_cluster_addr) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster_addr)
+               : "memory");
+}
+
+// Gathers, for a group of GROUP_THREADS producer threads, `rows` rows of `chunks` 16-byte
+// chunks: `src_of(j, c)` gives the source of chunk c of block row j (nullptr = zero fill),
+// `dst_of(r, c)` its shared-memory destination.
+template <typename SrcF, typename DstF>
+__device__ __forceinline__ void gather_rows(uint32_t gtid, uint32_t rows, uint32_t chunks, SrcF src_of, DstF dst_of,
+                                            const void* dummy) {
+  const uint32_t n = rows * chunks;
+  for (uint32_t i = gtid; i < n; i += AttnCfg::GROUP_THREADS) {
+    const uint32_t r = i / chunks, c = i - r * chunks;
+    const void* src = src_of(r, c);
+    cp_async_16(dst_of(r, c), src ? src : dummy, src ? 16u : 0u);
+  }
+}
+
 __global__ void __launch_bounds__(AttnCfg::THREADS, 1) __cluster_dims__(2, 1, 1)
-sparse_mla_attn_kernel(const AttnParams p) {
+sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnParams p) {
   using C = AttnCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  int32_t* sel = reinterpret_cast<int32_t*>(smem + C::OFF_SEL);
+  int32_t* sel2 = reinterpret_cast<int32_t*>(smem + C::OFF_SEL);
+  float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
   int32_t* scan = reinterpret_cast<int32_t*>(smem + C::OFF_SCAN);
   int32_t* info = reinterpret_cast<int32_t*>(smem + C::OFF_INFO);
   const uint32_t bar0 = sbase + C::OFF_BAR;
-  auto kv_full = [&](int s) { return bar0 + 8u * s; };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
-  const uint32_t s_full = bar0 + 8u * (2 * C::STAGES);
-  const uint32_t s_empty = s_full + 8, p_full = s_full + 16, p_empty = s_full + 24;
-  const uint32_t q_full = s_full + 32, q_empty = s_full + 40, o_empty = s_full + 48;
-  auto info_full = [&](int i) { return s_full + 56 + 8u * i; };
-  auto info_empty = [&](int i) { return s_full + 72 + 8u * i; };
-  auto x_full = [&](int i) { return s_full + 88 + 8u * i; };
-  auto x_empty = [&](int i) { return s_full + 104 + 8u * i; };
-  const uint32_t mma_done = s_full + 120;
+  auto B = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  // local barriers (both CTAs)
+  auto info_full = [&](int i) { return B(0 + i); };
+  auto info_empty = [&](int i) { return B(2 + i); };
+  auto sb_empty = [&](int s) { return B(4 + s); };       // commit: logits operand stage consumed
+  auto vr_empty = [&](int s) { return B(7 + s); };       // commit: output operand stage consumed
+  const uint32_t q_tma = B(9);                           // this CTA's smem part of q landed (TMA)
+  const uint32_t q_empty = B(10);                        // commit: all logits MMAs of a query done
+  auto s_full = [&](int i) { return B(11 + i); };        // commit: logits buffer i ready
+  const uint32_t p_empty = B(13);                        // commit: output MMA that read P done
+  const uint32_t o_full = B(14);                         // commit: all output MMAs of a query done
+  auto pair_bar = [&](int w, int par) { return B(15 + 2 * w + par); };   // softmax warp pairs
+  // barriers of the even CTA, arrived on by both CTAs
+  auto sb_full2 = [&](int s) { return B(19 + s); };
+  auto vr_full2 = [&](int s) { return B(22 + s); };
+  const uint32_t q_full2 = B(24);
+  auto s_empty2 = [&](int i) { return B(25 + i); };
+  const uint32_t p_full2 = B(27);
+  const uint32_t o_empty2 = B(28);
+  const uint32_t mma_done = B(29);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
   const uint32_t warp = warp_id(), lane = lane_id();
   const uint32_t rank = cluster_ctarank();
-  const uint32_t peer = rank ^ 1u;
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(kv_full(s), C::PRODUCER_THREADS);
-      mbar_init(kv_empty(s), 1);
-    }
-    mbar_init(s_full, 1);
-    mbar_init(s_empty, C::SOFTMAX_WARPS);
-    mbar_init(p_full, C::SOFTMAX_WARPS);
-    mbar_init(p_empty, 1);
-    mbar_init(q_full, C::SOFTMAX_WARPS);
-    mbar_init(q_empty, 1);
-    mbar_init(o_empty, C::SOFTMAX_WARPS);
     for (int i = 0; i < 2; ++i) {
       mbar_init(info_full(i), 1);
-      mbar_init(info_empty(i), 1 + C::SOFTMAX_WARPS);
-      mbar_init(x_full(i), kHeads);     // arrived by the peer's 128 softmax threads
-      mbar_init(x_empty(i), kHeads);
+      // softmax warps + output-ring producer warps (+ the MMA thread in the even CTA)
+      mbar_init(info_empty(i), C::SOFTMAX_WARPS + 2 + (leader ? 1 : 0));
+      mbar_init(s_full(i), 1);
+      mbar_init(s_empty2(i), 2 * C::SOFTMAX_WARPS);
+      mbar_init(vr_empty(i), 1);
+      mbar_init(vr_full2(i), 2 * 2);
     }
+    for (int i = 0; i < C::SB_STAGES; ++i) {
+      mbar_init(sb_empty(i), 1);
+      mbar_init(sb_full2(i), 2 * 2);
+    }
+    mbar_init(q_tma, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(p_empty, 1);
+    mbar_init(o_full, 1);
+    for (int w = 0; w < 2; ++w)
+      for (int par = 0; par < 2; ++par) mbar_init(pair_bar(w, par), 2);
+    mbar_init(q_full2, 2 * (1 + C::PRODUCER_WARPS));
+    mbar_init(p_full2, 2 * C::SOFTMAX_WARPS);
+    mbar_init(o_empty2, 2 * C::SOFTMAX_WARPS);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == C::MMA_WARP) {
-    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
-    tmem_relinquish();
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
-  cluster_sync();            // the peer's barriers are initialised before any remote arrive
+  cluster_sync();            // both CTAs' barriers and TMEM exist before any remote traffic
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   Waiter wt{p.status, abort_flag, p.wait_budget_ns, 2u};
   const int32_t ncl = static_cast<int32_t>(nclusters_x());
   const int32_t cid = static_cast<int32_t>(cluster_id_x());
-  const int32_t a0 = 256 * static_cast<int32_t>(rank);          // first dim of this CTA's stage rows
+  // cluster address of the even CTA's copy of a local barrier (arrives from either CTA)
+  const uint32_t lead_off = mapa(bar0, 0) - bar0;
+  auto at_leader = [&](uint32_t local_bar) { return local_bar + lead_off; };
 
   if (warp >= C::SOFTMAX_WARPS && warp < C::MMA_WARP) {
-    // ================================================================ producers: index list + gathers
-    // bar.sync cannot time out, so all producer threads take the same path through named
-    // barrier 2: thread 0 alone waits on mbarriers and publishes the go / stop decision in
-    // a parity slot that every thread reads after the barrier.
+    // ================================================================ producers
+    // Group A (warps 4,5; TMEM lanes 0..63): index compaction, the q operand (TMA part and
+    // TMEM lanes 0..63), and the logits ring (this CTA's 32 rows of each block, all dims).
+    // Group B (warps 6,7; TMEM lanes 64..127): the duplicate q lanes and the output ring
+    // (all 64 rows of each block, the 256 output dims this CTA supplies).
+    // Each group waits for its own copies (cp.async.wait_group, one group behind) and
+    // announces a stage to the even CTA per warp; the rings are independent, so a stage is
+    // announced without waiting for the other ring (no cycle through the MMA order).
     const uint32_t ptid = threadIdx.x - C::SOFTMAX_WARPS * 32;
-    volatile int32_t* go = scan + 8;                  // two parity slots
-    const int32_t nch = rank == 0 ? 36 : 40;          // 16-byte chunks per gathered row
-    const int32_t per = (p.topk + C::PRODUCER_THREADS - 1) / C::PRODUCER_THREADS;
-    uint32_t stage = 0, phase = 0, qn = 0, nsync = 0;
-    auto gate = [&](uint32_t bar, uint32_t parity, uint32_t tag) -> bool {
-      if (ptid == 0) go[nsync & 1u] = wt.wait(bar, parity, tag) ? 1 : 0;
-      named_barrier(2, C::PRODUCER_THREADS);
+    const uint32_t pw = ptid >> 5;                     // 0..3 = TMEM lane quarter
+    const bool group_a = pw < 2;
+    const uint32_t gtid = ptid & 63u;
+    volatile int32_t* go = scan + 8;
+    const int32_t per = (p.topk + C::GROUP_THREADS - 1) / C::GROUP_THREADS;
+    uint32_t qn = 0, nsync = 0, qq = 0;
+    uint32_t st = 0, ph = 0;                            // ring position (this group's ring)
+    const uint32_t n_stages = group_a ? C::SB_STAGES : C::VR_STAGES;
+    bool ok = true;
+    auto gate = [&](uint32_t bar, uint32_t parity, uint32_t tag) -> bool {   // group A only
+      if (gtid == 0) go[nsync & 1u] = (wt.wait(bar, parity, tag) && !wt.aborted()) ? 1 : 0;
+      named_barrier(2, C::GROUP_THREADS);
       return go[(nsync++) & 1u] != 0;
+    };
+    auto warp_wait = [&](uint32_t bar, uint32_t parity, uint32_t tag) -> bool {
+      uint32_t got = 1;
+      if (lane == 0) got = wt.wait(bar, parity, tag) ? 1u : 0u;
+      return __shfl_sync(0xffffffffu, got, 0) != 0;
     };
     for (int32_t qi = cid; qi < p.n_queries; qi += ncl, ++qn) {
       const uint32_t slot = qn & 1u, sph = (qn >> 1) & 1u;
-      if (!gate(info_empty(slot), sph ^ 1u, 10)) break;
-      // compact the valid entries of the index row, preserving their order
-      const int32_t* row = p.idx + static_cast<size_t>(qi) * p.topk;
-      const int32_t j0 = min(static_cast<int32_t>(ptid) * per, p.topk), j1 = min(j0 + per, p.topk);
-      int32_t cnt = 0;
-      for (int32_t j = j0; j < j1; ++j) {
-        const int32_t v = __ldg(row + j);
-        if (v >= p.max_len) record_error(p.status, DSA_ERR_INDEX_RANGE, static_cast<uint32_t>(qi));
-        cnt += (v >= 0 && v < p.max_len) ? 1 : 0;
-      }
-      int32_t incl = cnt;
+      int32_t* sel = sel2 + slot * kMaxTopk;
+      int32_t total = 0;
+      if (group_a) {
+        if (!gate(info_empty(slot), sph ^ 1u, 10)) break;
+        // ---- compact the valid entries of the index row, preserving their order
+        const int32_t* row = p.idx + static_cast<size_t>(qi) * p.topk;
+        const int32_t j0 = min(static_cast<int32_t>(gtid) * per, p.topk), j1 = min(j0 + per, p.topk);
+        int32_t cnt = 0;
+        for (int32_t j = j0; j < j1; ++j) {
+          const int32_t v = __ldg(row + j);
+          if (v >= p.max_len) record_error(p.status, DSA_ERR_INDEX_RANGE, static_cast<uint32_t>(qi));
+          cnt += (v >= 0 && v < p.max_len) ? 1 : 0;
+        }
+        int32_t incl = cnt;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (static_cast<int32_t>(lane) >= o) incl += v;
-      }
-      if (lane == 31) scan[ptid >> 5] = incl;
-      named_barrier(2, C::PRODUCER_THREADS);
-      int32_t base = incl - cnt, total = 0;
-      for (uint32_t w = 0; w < C::PRODUCER_WARPS; ++w) {
-        const int32_t v = scan[w];
-        if (w < (ptid >> 5)) base += v;
-        total += v;
-      }
-      for (int32_t j = j0; j < j1; ++j) {
-        const int32_t v = __ldg(row + j);
-        if (v >= 0 && v < p.max_len) sel[base++] = v;
-      }
-      named_barrier(2, C::PRODUCER_THREADS);
-      if (ptid == 0) {
-        info[slot] = total;
-        mbar_arrive(info_full(slot));
+        for (int o = 1; o < 32; o <<= 1) {
+          const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (static_cast<int32_t>(lane) >= o) incl += v;
+        }
+        if (lane == 31) scan[pw] = incl;
+        named_barrier(2, C::GROUP_THREADS);
+        int32_t base = incl - cnt + (pw == 1 ? scan[0] : 0);
+        total = scan[0] + scan[1];
+        for (int32_t j = j0; j < j1; ++j) {
+          const int32_t v = __ldg(row + j);
+          if (v >= 0 && v < p.max_len) sel[base++] = v;
+        }
+        named_barrier(2, C::GROUP_THREADS);
+        if (gtid == 0) {
+          info[slot] = total;
+          mbar_arrive(info_full(slot));
+        }
+      } else {
+        if (!warp_wait(info_full(slot), sph, 14)) break;
+        total = info[slot];
       }
       const int32_t n_blocks = (total + kBlk - 1) / kBlk;
-      const size_t kv_seq = static_cast<size_t>(qi / p.n_q) * p.max_len;
-      int32_t pending_stage = -1;
-      bool ok = true;
-      for (int32_t b = 0; b < n_blocks; ++b) {
-        if (!gate(kv_empty(stage), phase ^ 1u, 11)) { ok = false; break; }
-        const uint32_t st = sbase + C::OFF_STAGE + stage * C::STAGE_BYTES;
-        for (int32_t i = ptid; i < kBlk * nch; i += C::PRODUCER_THREADS) {
-          const int32_t r = i / nch, ch = i - r * nch;
-          const int32_t j = b * kBlk + r;
-          const bool valid = j < total;
-          const __nv_bfloat16* src = p.kv;
-          if (valid) src = p.kv + (kv_seq + sel[j]) * kDqk + a0 + ch * 8;
-          const uint32_t dst = st + (ch >> 3) * C::ATOM_BYTES + sw128_offset(r, ch & 7);
-          cp_async_16(dst, src, valid ? 16u : 0u);
+      if (n_blocks > 0 && ok) {
+        // ---- the q operand: dims 384..575 by TMA into shared memory (group A thread 0),
+        // dims 0..383 into TMEM lanes of this warp (both lane halves: the same 64 heads)
+        if (warp_wait(q_empty, (qq & 1u) ^ 1u, 12)) {
+          if (ptid == 0) {
+            mbar_expect_tx(q_tma, C::QS_BYTES);
+            for (int a = 0; a < C::QS_ATOMS; ++a)
+              tma_load_3d(sbase + C::OFF_QS + a * 8192, &map_q, q_tma, C::Q_TMEM_DIMS + 64 * a,
+                          qi * kHeads + 64 * static_cast<int32_t>(rank), 0);
+          }
+          tc_fence_after();
+          const uint32_t hl = ptid & 63u;
+          const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(qi) * kHeads + 64 * rank + hl) *
+                                                             kDqk);
+#pragma unroll 1
+          for (int c = 0; c < C::Q_TMEM_DIMS / 32; ++c) {     // 16 columns (32 dims) at a time
+            uint32_t r[16];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint4 u = __ldg(qsrc + c * 4 + v);
+              r[4 * v + 0] = u.x; r[4 * v + 1] = u.y; r[4 * v + 2] = u.z; r[4 * v + 3] = u.w;
+            }
+            tmem_st16(tmem + ((pw * 32u) << 16) + C::COL_Q + 16 * c, r);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(at_leader(q_full2));
+          if (ptid == 0 && wt.wait(q_tma, qq & 1u, 13)) mbar_arrive_cluster(at_leader(q_full2));
+        } else {
+          ok = false;
         }
-        cp_async_commit();
-        if (pending_stage >= 0) {
-          cp_async_wait<1>();
+        ++qq;
+        // ---- the ring of this group
+        const size_t kv_seq = static_cast<size_t>(qi / p.n_q) * p.max_len;
+        const int32_t own0 = 32 * static_cast<int32_t>(rank);
+        int32_t pending = -1;
+        for (int32_t b = 0; b < n_blocks && ok; ++b) {
+          if (!warp_wait(group_a ? sb_empty(st) : vr_empty(st), ph ^ 1u, 11)) { ok = false; break; }
+          if (group_a) {
+            const uint32_t sb = sbase + C::OFF_SB + st * C::SB_BYTES;
+            gather_rows(
+                gtid, 32, 72,
+                [&](uint32_t r, uint32_t c) -> const void* {
+                  const int32_t j = b * kBlk + own0 + static_cast<int32_t>(r);
+                  return j < total ? static_cast<const void*>(p.kv + (kv_seq + sel[j]) * kDqk + c * 8) : nullptr;
+                },
+                [&](uint32_t r, uint32_t c) { return sb + (c >> 3) * C::SB_ATOM + sw128_offset(r, c & 7u); }, p.kv);
+          } else {
+            const uint32_t vr = sbase + C::OFF_VR + st * C::VR_BYTES;
+            gather_rows(
+                gtid, kBlk, 32,
+                [&](uint32_t r, uint32_t c) -> const void* {
+                  const int32_t j = b * kBlk + static_cast<int32_t>(r);
+                  const uint32_t slot4 = c >> 3;
+                  const uint32_t atom = 4 * (slot4 >> 1) + 2 * rank + (slot4 & 1u);
+                  return j < total ? static_cast<const void*>(p.kv + (kv_seq + sel[j]) * kDqk + atom * 64 + (c & 7u) * 8)
+                                   : nullptr;
+                },
+                [&](uint32_t r, uint32_t c) { return vr + (c >> 3) * C::VR_ATOM + sw128_offset(r, c & 7u); }, p.kv);
+          }
+          cp_async_commit();
+          if (pending >= 0) {
+            cp_async_wait<1>();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(at_leader(group_a ? sb_full2(pending) : vr_full2(pending)));
+          }
+          pending = static_cast<int32_t>(st);
+          if (++st == n_stages) { st = 0; ph ^= 1u; }
+        }
+        cp_async_wait<0>();
+        if (pending >= 0) {
           fence_proxy_async_smem();
-          mbar_arrive(kv_full(pending_stage));
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(at_leader(group_a ? sb_full2(pending) : vr_full2(pending)));
         }
-        pending_stage = static_cast<int32_t>(stage);
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
       }
-      cp_async_wait<0>();
-      if (pending_stage >= 0) {
-        fence_proxy_async_smem();
-        mbar_arrive(kv_full(pending_stage));
+      if (!group_a) {                                  // sel[slot] no longer read by this warp
+        __syncwarp();
+        if (lane == 0) mbar_arrive(info_empty(slot));
       }
-      if (!ok) break;
     }
     cp_async_wait<0>();
   } else if (warp == C::MMA_WARP) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
+    // ================================================================ MMA issuer (even CTA only)
+    if (leader && lane == 0) {
       constexpr uint32_t idesc_s = make_idesc(1, 1, 0, 0, 128, kBlk);
-      constexpr uint32_t idesc_pv = make_idesc(1, 1, 0, 1, 128, 256);
-      uint32_t stage = 0, phase = 0, qn = 0, sb = 0, pb = 0, qq = 0;
-      for (int32_t qi = cid; qi < p.n_queries; qi += ncl, ++qn) {
-        const uint32_t slot = qn & 1u, sph = (qn >> 1) & 1u;
-        if (!wt.wait(info_full(slot), sph, 20)) break;
+      constexpr uint32_t idesc_o = make_idesc(1, 1, 0, 1, 128, 256);
+      const uint32_t peer_off = mapa(bar0, 1) - bar0;
+      auto commit_both = [&](uint32_t local_bar) {
+        commit2(local_bar);
+        commit2(local_bar + peer_off);
+      };
+      uint32_t sst = 0, sph = 0, vst = 0, vph = 0, qn = 0, sb = 0, pb = 0, qq = 0;
+      bool ok = true;
+      for (int32_t qi = cid; qi < p.n_queries && ok; qi += ncl, ++qn) {
+        const uint32_t slot = qn & 1u, iph = (qn >> 1) & 1u;
+        if (!wt.wait(info_full(slot), iph, 20)) break;
         const int32_t total = info[slot];
         mbar_arrive(info_empty(slot));
         const int32_t n_blocks = (total + kBlk - 1) / kBlk;
         if (n_blocks == 0) continue;
-        if (!wt.wait(q_full, qq & 1u, 21)) break;
-        bool ok = true;
-        // logits of block 0, then per block: logits of block b+1, then P.V of block b
-        const uint32_t s_stage = stage, s_phase = phase;
-        auto do_s = [&](uint32_t stg, uint32_t ph) -> bool {
-          if (!wt.wait(kv_full(stg), ph, 22)) return false;
-          if (!wt.wait(s_empty, (sb & 1u) ^ 1u, 23)) return false;
+        if (!wt.wait(q_full2, qq & 1u, 21)) break;
+        // logits of the next block into TMEM buffer sb&1 from the next logits stage
+        auto do_s = [&]() -> bool {
+          if (!wt.wait(sb_full2(sst), sph, 22)) return false;
+          if (!wt.wait(s_empty2(sb & 1u), ((sb >> 1) & 1u) ^ 1u, 23)) return false;
           tc_fence_after();
-          const uint32_t st = sbase + C::OFF_STAGE + stg * C::STAGE_BYTES;
+          const uint32_t sbuf = sbase + C::OFF_SB + sst * C::SB_BYTES;
+          const uint32_t d = tmem + C::COL_S + 32u * (sb & 1u);
 #pragma unroll
-          for (int j = 0; j < 18; ++j) {
-            const int dj = (rank == 0 ? 0 : 32) + 16 * j;
-            const uint32_t addr = st + (dj >> 6) * C::ATOM_BYTES + (dj & 63) * 2;
-            mma_bf16_ts(tmem + C::COL_S, tmem + C::COL_Q + 8 * j, sw128_desc(addr, 1, 1024), idesc_s,
-                        j > 0 ? 1u : 0u);
+          for (int j = 0; j < C::Q_TMEM_DIMS / 16; ++j) {      // A from TMEM
+            const int dj = 16 * j;
+            mma2_ts(d, tmem + C::COL_Q + 8 * j, sw128_desc(sbuf + (dj >> 6) * C::SB_ATOM + (dj & 63) * 2, 1, 1024),
+                    idesc_s, j > 0 ? 1u : 0u);
           }
-          tc_commit(s_full);
+#pragma unroll
+          for (int j = C::Q_TMEM_DIMS / 16; j < kDqk / 16; ++j) {   // A from shared memory
+            const int dj = 16 * j, dq = dj - C::Q_TMEM_DIMS;
+            mma2_ss(d, sw128_desc(sbase + C::OFF_QS + (dq >> 6) * 8192 + (dq & 63) * 2, 1, 1024),
+                    sw128_desc(sbuf + (dj >> 6) * C::SB_ATOM + (dj & 63) * 2, 1, 1024), idesc_s, 1u);
+          }
+          commit_both(s_full(sb & 1u));
+          commit_both(sb_empty(sst));
           ++sb;
+          if (++sst == C::SB_STAGES) { sst = 0; sph ^= 1u; }
           return true;
         };
-        if (!do_s(s_stage, s_phase)) break;
+        if (!do_s()) break;
         for (int32_t b = 0; b < n_blocks; ++b) {
-          const uint32_t cur_stage = stage;
-          uint32_t nstage = stage + 1, nphase = phase;
-          if (nstage == C::STAGES) { nstage = 0; nphase ^= 1u; }
           if (b + 1 < n_blocks) {
-            if (!do_s(nstage, nphase)) { ok = false; break; }
+            if (!do_s()) { ok = false; break; }
+          } else {
+            commit_both(q_empty);                  // every logits MMA of the query is issued
           }
-          if (!wt.wait(p_full, pb & 1u, 24)) { ok = false; break; }
-          if (b == 0 && !wt.wait(o_empty, (qq & 1u) ^ 1u, 25)) { ok = false; break; }
+          if (!wt.wait(vr_full2(vst), vph, 26)) { ok = false; break; }
+          if (!wt.wait(p_full2, pb & 1u, 24)) { ok = false; break; }
+          if (b == 0 && !wt.wait(o_empty2, (qq & 1u) ^ 1u, 25)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t st = sbase + C::OFF_STAGE + cur_stage * C::STAGE_BYTES;
+          const uint32_t vr = sbase + C::OFF_VR + vst * C::VR_BYTES;
+          const uint32_t pbuf = sbase + C::OFF_P;
 #pragma unroll
-          for (int kk = 0; kk < kBlk / 16; ++kk) {
-            mma_bf16_ts(tmem + C::COL_O, tmem + C::COL_P + 8 * kk,
-                        sw128_desc(st + kk * 2048, C::ATOM_BYTES, 1024), idesc_pv, (b > 0 || kk > 0) ? 1u : 0u);
+          for (int i = 0; i < 2; ++i) {
+#pragma unroll
+            for (int kk = 0; kk < kBlk / 16; ++kk) {
+              mma2_ss(tmem + C::COL_O + 128 * i, sw128_desc(pbuf + kk * 32, 1, 1024),
+                      sw128_desc(vr + 2 * i * C::VR_ATOM + kk * 2048, C::VR_ATOM, 1024), idesc_o,
+                      (b > 0 || kk > 0) ? 1u : 0u);
+            }
           }
-          tc_commit(kv_empty(cur_stage));
-          tc_commit(p_empty);
+          commit_both(vr_empty(vst));
+          commit_both(p_empty);
           ++pb;
-          stage = nstage;
-          phase = nphase;
+          if (++vst == C::VR_STAGES) { vst = 0; vph ^= 1u; }
         }
-        tc_commit(q_empty);
-        ++qq;
         if (!ok) break;
+        commit_both(o_full);
+        ++qq;
       }
       tc_commit(mma_done);
       attn_drain_wait(mma_done, 0, p.wait_budget_ns);
     }
   } else {
-    // ================================================================ softmax / epilogue warps (thread = head)
-    const uint32_t h = threadIdx.x;                  // 0..127, TMEM lane h
+    // ================================================================ softmax warps (TMEM lane = thread)
+    // lane L: head 64*rank + (L % 64); logits of block rows 32*(L/64) .. +31; output dims
+    // 256 i + 128 (L/64) .. +127 for i = 0, 1. Warps w and w+2 hold the two halves of the
+    // same 32 heads and exchange row maxima (and, at the end, row sums) in shared memory.
+    const uint32_t L = threadIdx.x;
+    const uint32_t half = L >> 6;
+    const uint32_t hl = L & 63u;
     const uint32_t lane_off = (warp * 32u) << 16;
-    const uint32_t xpeer = mapa(sbase + C::OFF_X, peer);
-    const uint32_t xfull_peer0 = mapa(x_full(0), peer);
-    const uint32_t xempty_peer0 = mapa(x_empty(0), peer);
-    const float* xloc = reinterpret_cast<const float*>(smem + C::OFF_X);
-    uint32_t qn = 0, sb = 0, pb = 0, qq = 0, xb = 0;
+    const uint32_t pairw = warp & 1u;                  // warps 0,2 -> pair 0; 1,3 -> pair 1
+    const uint32_t partner = L ^ 64u;
+    uint32_t qn = 0, sb = 0, pb = 0, nx = 0, qd = 0;
     bool ok = true;
+    // one float from the partner lane (the other half of the same head)
+    auto swap_partner = [&](float mine) -> float {
+      const uint32_t par = nx & 1u, ph = (nx >> 1) & 1u;
+      ++nx;
+      xmax[par * 128 + L] = mine;
+      __syncwarp();
+      uint32_t got = 1;
+      if (lane == 0) {
+        mbar_arrive(pair_bar(pairw, par));
+        got = wt.wait(pair_bar(pairw, par), ph, 37) ? 1u : 0u;
+      }
+      if (!__shfl_sync(0xffffffffu, got, 0)) ok = false;
+      return xmax[par * 128 + partner];
+    };
     for (int32_t qi = cid; qi < p.n_queries && ok; qi += ncl, ++qn) {
       const uint32_t slot = qn & 1u, sph = (qn >> 1) & 1u;
       uint32_t got = 1;
@@ -313,88 +487,37 @@ sparse_mla_attn_kernel(const AttnParams p) {
       __syncwarp();
       if (lane == 0) mbar_arrive(info_empty(slot));
       const int32_t n_blocks = (total + kBlk - 1) / kBlk;
-      __nv_bfloat16* orow = p.out + (static_cast<size_t>(qi) * kHeads + h) * kDv + 256 * rank;
+      const size_t orow = (static_cast<size_t>(qi) * kHeads + 64 * rank + hl) * kDv;
       if (n_blocks == 0) {
-        const uint4 z = make_uint4(0, 0, 0, 0);
-        for (int c = 0; c < 32; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
-        if (rank == 0) p.lse[static_cast<size_t>(qi) * kHeads + h] = -INFINITY;
+        const uint4 zz = make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 2; ++i)
+          for (int c = 0; c < 16; ++c) reinterpret_cast<uint4*>(p.out + orow + 256 * i + 128 * half)[c] = zz;
+        if (half == 0) p.lse[static_cast<size_t>(qi) * kHeads + 64 * rank + hl] = -INFINITY;
         continue;
       }
-      // ---- Q[:, 288r : 288r+288] -> TMEM columns COL_Q.. (A operand of the logits MMA)
-      if (lane == 0) got = wt.wait(q_empty, (qq & 1u) ^ 1u, 31) ? 1u : 0u;
-      if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
-      tc_fence_after();
-      {
-        const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(qi) * kHeads + h) * kDqk +
-                                                           288 * rank);
-#pragma unroll 1
-        for (int c = 0; c < 9; ++c) {          // 9 x 16 columns = 288 bf16
-          uint32_t r[16];
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint4 u = __ldg(qsrc + c * 4 + v);
-            r[4 * v + 0] = u.x; r[4 * v + 1] = u.y; r[4 * v + 2] = u.z; r[4 * v + 3] = u.w;
-          }
-          tmem_st16(tmem + lane_off + C::COL_Q + 16 * c, r);
-        }
-        tmem_wait_st();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(q_full);
-      ++qq;
       float m2 = -INFINITY, l = 0.f;
-      for (int32_t b = 0; b < n_blocks; ++b) {
-        // ---- partial logits from TMEM
-        if (lane == 0) got = wt.wait(s_full, sb & 1u, 32) ? 1u : 0u;
+      for (int32_t b = 0; b < n_blocks && ok; ++b) {
+        // ---- this lane's 32 logits
+        if (lane == 0) got = wt.wait(s_full(sb & 1u), (sb >> 1) & 1u, 32) ? 1u : 0u;
         if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sr[64];
-        tmem_ld32(tmem + lane_off + C::COL_S, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(tmem + lane_off + C::COL_S + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        uint32_t sr[32];
+        tmem_ld32(tmem + lane_off + C::COL_S + 32u * (sb & 1u), sr);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_empty);
+        if (lane == 0) mbar_arrive_cluster(at_leader(s_empty2(sb & 1u)));
         ++sb;
-        // ---- swap partials with the peer CTA (distributed shared memory)
-        const uint32_t xs = xb & 1u, xph = (xb >> 1) & 1u;
-        ++xb;
-        if (!wt.wait<true>(x_empty(xs), xph ^ 1u, 33)) { ok = false; break; }
-        {
-          const uint32_t rowaddr = xpeer + xs * C::X_BYTES + h * 256u;
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            st_cluster_v4(rowaddr + ((c ^ (h & 15u)) << 4), __uint_as_float(sr[4 * c]), __uint_as_float(sr[4 * c + 1]),
-                          __uint_as_float(sr[4 * c + 2]), __uint_as_float(sr[4 * c + 3]));
-          }
-        }
-        mbar_arrive_cluster(xfull_peer0 + 8u * xs);
-        if (!wt.wait<true>(x_full(xs), xph, 34)) { ok = false; break; }
-        float z[64];
-        {
-          const float* rowp = xloc + xs * (C::X_BYTES / 4) + h * 64u;
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float4 o = *reinterpret_cast<const float4*>(rowp + ((c ^ (h & 15u)) << 2));
-            const float m0 = __uint_as_float(sr[4 * c]), m1 = __uint_as_float(sr[4 * c + 1]);
-            const float m2_ = __uint_as_float(sr[4 * c + 2]), m3 = __uint_as_float(sr[4 * c + 3]);
-            // fixed order (rank-0 partial + rank-1 partial): both CTAs get identical sums
-            z[4 * c + 0] = rank == 0 ? m0 + o.x : o.x + m0;
-            z[4 * c + 1] = rank == 0 ? m1 + o.y : o.y + m1;
-            z[4 * c + 2] = rank == 0 ? m2_ + o.z : o.z + m2_;
-            z[4 * c + 3] = rank == 0 ? m3 + o.w : o.w + m3;
-          }
-        }
-        mbar_arrive_cluster(xempty_peer0 + 8u * xs);
-        // ---- online softmax (log2 domain), lazy rescale
-        const int32_t nvalid = min(kBlk, total - b * kBlk);
+        const int32_t nvalid = min(32, total - b * kBlk - 32 * static_cast<int32_t>(half));
+        float z[32];
         float mb = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          z[j] = (j < nvalid) ? z[j] * p.scale_log2 : -INFINITY;
+        for (int j = 0; j < 32; ++j) {
+          z[j] = (j < nvalid) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
           mb = fmaxf(mb, z[j]);
         }
+        mb = fmaxf(mb, swap_partner(mb));
+        if (!ok) break;
         const bool need = (mb > m2 + 8.0f);
         float alpha = 1.0f;
         if (need) {
@@ -402,80 +525,93 @@ sparse_mla_attn_kernel(const AttnParams p) {
           m2 = mb;
           l *= alpha;
         }
-        uint32_t pk[32];
+        uint32_t pk[16];
         float lsum = 0.f;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 16; ++j) {
           const __nv_bfloat162 pr = __floats2bfloat162_rn(ex2_approx(z[2 * j] - m2), ex2_approx(z[2 * j + 1] - m2));
           const float2 back = __bfloat1622float2(pr);
           lsum += back.x + back.y;
           pk[j] = *reinterpret_cast<const uint32_t*>(&pr);
         }
         l += lsum;
-        // ---- P -> TMEM (and rescale O) once the previous P.V has finished
-        if (b > 0) {
-          if (lane == 0) got = wt.wait(p_empty, (pb & 1u), 35) ? 1u : 0u;
+        // ---- the P buffer is free, and O stable, once the previous output MMA has finished
+        if (pb >= 1) {
+          if (lane == 0) got = wt.wait(p_empty, (pb - 1) & 1u, 35) ? 1u : 0u;
           if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
-          ++pb;
+        }
+        // ---- rescale this lane's output columns if the running max moved
+        if (__any_sync(0xffffffffu, need) && b > 0) {
           tc_fence_after();
-          if (__any_sync(0xffffffffu, need)) {
-            const float a = need ? alpha : 1.0f;
+          const float a = need ? alpha : 1.0f;
 #pragma unroll 1
-            for (int c = 0; c < 16; ++c) {
-              uint32_t o[16];
-              tmem_ld16(tmem + lane_off + C::COL_O + 16 * c, o);
-              tmem_wait_ld();
+          for (int c = 0; c < 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tmem + lane_off + C::COL_O + 16 * c, o);
+            tmem_wait_ld();
 #pragma unroll
-              for (int v = 0; v < 16; ++v) o[v] = __float_as_uint(__uint_as_float(o[v]) * a);
-              tmem_st16(tmem + lane_off + C::COL_O + 16 * c, o);
-            }
+            for (int v = 0; v < 16; ++v) o[v] = __float_as_uint(__uint_as_float(o[v]) * a);
+            tmem_st16(tmem + lane_off + C::COL_O + 16 * c, o);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+        }
+        {
+          // P row hl, columns 32*half .. +31 (64 B = 4 chunks of the 128-byte swizzled row)
+          const uint32_t prow = sbase + C::OFF_P;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(prow + sw128_offset(hl, 4 * half + c)),
+                         "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                         : "memory");
           }
         }
-        tmem_st16(tmem + lane_off + C::COL_P, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-        tmem_st16(tmem + lane_off + C::COL_P + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
-        tmem_wait_st();
-        tc_fence_before();
+        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive_cluster(at_leader(p_full2));
+        ++pb;
       }
       if (!ok) break;
-      // ---- epilogue: wait for the last P.V, normalise, store
-      if (lane == 0) got = wt.wait(p_empty, (pb & 1u), 36) ? 1u : 0u;
+      // ---- epilogue: row sum of both halves, wait for the last output MMA, normalise, store
+      l += swap_partner(l);
+      if (!ok) break;
+      if (lane == 0) got = wt.wait(o_full, qd & 1u, 36) ? 1u : 0u;
       if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
-      ++pb;
+      ++qd;
       tc_fence_after();
       const float inv = 1.0f / l;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 8; ++c) {               // 2 instructions x 128 columns, 32 at a time
         uint32_t o[32];
         tmem_ld32(tmem + lane_off + C::COL_O + 32 * c, o);
         tmem_wait_ld();
         uint4 pkd[4];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
+        uint32_t* pw32 = reinterpret_cast<uint32_t*>(pkd);
 #pragma unroll
         for (int v = 0; v < 16; ++v) {
           const __nv_bfloat162 pr =
               __floats2bfloat162_rn(__uint_as_float(o[2 * v]) * inv, __uint_as_float(o[2 * v + 1]) * inv);
-          pw[v] = *reinterpret_cast<const uint32_t*>(&pr);
+          pw32[v] = *reinterpret_cast<const uint32_t*>(&pr);
         }
-        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+        const int i = c >> 2, cc = c & 3;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + orow + 256 * i + 128 * half + 32 * cc);
 #pragma unroll
         for (int v = 0; v < 4; ++v) dst[v] = pkd[v];
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_empty);
-      if (rank == 0) p.lse[static_cast<size_t>(qi) * kHeads + h] = (m2 + log2f(l)) * 0.69314718055994531f;
+      if (lane == 0) mbar_arrive_cluster(at_leader(o_empty2));
+      if (half == 0) p.lse[static_cast<size_t>(qi) * kHeads + 64 * rank + hl] = (m2 + log2f(l)) * 0.69314718055994531f;
     }
   }
   // ---- teardown: every role reaches here (all waits are bounded)
   tc_fence_before();
   __syncthreads();
-  cluster_sync();            // no CTA leaves while its peer may still touch its shared memory
+  cluster_sync();            // no CTA leaves while its peer may still use its memory
   if (warp == C::MMA_WARP) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS) : "memory");
   }
 }
 
