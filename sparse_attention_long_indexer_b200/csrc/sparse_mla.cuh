@@ -123,20 +123,6 @@ __device__ __forceinline__ void commit2(uint32_t bar_cluster_addr) {
                : "memory");
 }
 
-// Gathers, for a group of GROUP_THREADS producer threads, `rows` rows of `chunks` 16-byte
-// chunks: `src_of(j, c)` gives the source of chunk c of block row j (nullptr = zero fill),
-// `dst_of(r, c)` its shared-memory destination.
-template <typename SrcF, typename DstF>
-__device__ __forceinline__ void gather_rows(uint32_t gtid, uint32_t rows, uint32_t chunks, SrcF src_of, DstF dst_of,
-                                            const void* dummy) {
-  const uint32_t n = rows * chunks;
-  for (uint32_t i = gtid; i < n; i += AttnCfg::GROUP_THREADS) {
-    const uint32_t r = i / chunks, c = i - r * chunks;
-    const void* src = src_of(r, c);
-    cp_async_16(dst_of(r, c), src ? src : dummy, src ? 16u : 0u);
-  }
-}
-
 __global__ void __launch_bounds__(AttnCfg::THREADS, 1) __cluster_dims__(2, 1, 1)
 sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnParams p) {
   using C = AttnCfg;
@@ -321,50 +307,76 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
           ok = false;
         }
         ++qq;
-        // ---- the ring of this group
-        const size_t kv_seq = static_cast<size_t>(qi / p.n_q) * p.max_len;
+        // ---- the ring of this group. Thread (r0, cc) copies 16-byte chunk cc of every 128-byte
+        // segment of block rows r0, r0 + 8, ...: the row indices are read once per block and each
+        // copy is a constant offset from the row's base, so copies issue back to back.
+        const __nv_bfloat16* kv_seq = p.kv + static_cast<size_t>(qi / p.n_q) * p.max_len * kDqk;
+        const uint32_t cc = gtid & 7u, r0 = gtid >> 3;
         const int32_t own0 = 32 * static_cast<int32_t>(rank);
+        const uint32_t seg0 = 128u * rank;               // group B: segments 2r, 2r+1, 4+2r, 5+2r
         int32_t pending = -1;
+        auto announce = [&](int32_t stage) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(at_leader(group_a ? sb_full2(stage) : vr_full2(stage)));
+        };
         for (int32_t b = 0; b < n_blocks && ok; ++b) {
-          if (!warp_wait(group_a ? sb_empty(st) : vr_empty(st), ph ^ 1u, 11)) { ok = false; break; }
+          const uint32_t empty_bar = group_a ? sb_empty(st) : vr_empty(st);
+          if (pending >= 0) {                          // about to wait: announce the last stage first
+            uint32_t free_now = 0;
+            if (lane == 0) free_now = mbar_test_wait(empty_bar, ph ^ 1u) ? 1u : 0u;
+            if (!__shfl_sync(0xffffffffu, free_now, 0)) {
+              cp_async_wait<0>();
+              announce(pending);
+              pending = -1;
+            }
+          }
+          if (!warp_wait(empty_bar, ph ^ 1u, 11)) { ok = false; break; }
           if (group_a) {
-            const uint32_t sb = sbase + C::OFF_SB + st * C::SB_BYTES;
-            gather_rows(
-                gtid, 32, 72,
-                [&](uint32_t r, uint32_t c) -> const void* {
-                  const int32_t j = b * kBlk + own0 + static_cast<int32_t>(r);
-                  return j < total ? static_cast<const void*>(p.kv + (kv_seq + sel[j]) * kDqk + c * 8) : nullptr;
-                },
-                [&](uint32_t r, uint32_t c) { return sb + (c >> 3) * C::SB_ATOM + sw128_offset(r, c & 7u); }, p.kv);
+            const uint32_t dst0 = sbase + C::OFF_SB + st * C::SB_BYTES + sw128_offset(r0, cc);
+            int32_t rows[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int32_t j = b * kBlk + own0 + static_cast<int32_t>(r0) + 8 * q;
+              rows[q] = j < total ? sel[j] : -1;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const bool v = rows[q] >= 0;
+              const __nv_bfloat16* src = (v ? kv_seq + static_cast<size_t>(rows[q]) * kDqk : p.kv) + cc * 8;
+              const uint32_t n = v ? 16u : 0u;
+#pragma unroll
+              for (int a = 0; a < 9; ++a) cp_async_16(dst0 + q * 1024 + a * C::SB_ATOM, src + a * 64, n);
+            }
           } else {
-            const uint32_t vr = sbase + C::OFF_VR + st * C::VR_BYTES;
-            gather_rows(
-                gtid, kBlk, 32,
-                [&](uint32_t r, uint32_t c) -> const void* {
-                  const int32_t j = b * kBlk + static_cast<int32_t>(r);
-                  const uint32_t slot4 = c >> 3;
-                  const uint32_t atom = 4 * (slot4 >> 1) + 2 * rank + (slot4 & 1u);
-                  return j < total ? static_cast<const void*>(p.kv + (kv_seq + sel[j]) * kDqk + atom * 64 + (c & 7u) * 8)
-                                   : nullptr;
-                },
-                [&](uint32_t r, uint32_t c) { return vr + (c >> 3) * C::VR_ATOM + sw128_offset(r, c & 7u); }, p.kv);
+            const uint32_t dst0 = sbase + C::OFF_VR + st * C::VR_BYTES + sw128_offset(r0, cc);
+            int32_t rows[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int32_t j = b * kBlk + static_cast<int32_t>(r0) + 8 * q;
+              rows[q] = j < total ? sel[j] : -1;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const bool v = rows[q] >= 0;
+              const __nv_bfloat16* src = (v ? kv_seq + static_cast<size_t>(rows[q]) * kDqk : p.kv) + seg0 + cc * 8;
+              const uint32_t n = v ? 16u : 0u;
+              cp_async_16(dst0 + q * 1024 + 0 * C::VR_ATOM, src + 0, n);
+              cp_async_16(dst0 + q * 1024 + 1 * C::VR_ATOM, src + 64, n);
+              cp_async_16(dst0 + q * 1024 + 2 * C::VR_ATOM, src + 256, n);
+              cp_async_16(dst0 + q * 1024 + 3 * C::VR_ATOM, src + 320, n);
+            }
           }
           cp_async_commit();
           if (pending >= 0) {
             cp_async_wait<1>();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(at_leader(group_a ? sb_full2(pending) : vr_full2(pending)));
+            announce(pending);
           }
           pending = static_cast<int32_t>(st);
           if (++st == n_stages) { st = 0; ph ^= 1u; }
         }
         cp_async_wait<0>();
-        if (pending >= 0) {
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(at_leader(group_a ? sb_full2(pending) : vr_full2(pending)));
-        }
+        if (pending >= 0) announce(pending);
       }
       if (!group_a) {                                  // sel[slot] no longer read by this warp
         __syncwarp();
