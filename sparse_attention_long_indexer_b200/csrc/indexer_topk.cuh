@@ -41,9 +41,9 @@ constexpr int kDecodeChunk = 8192;  // keys per decode work item
 template <int NQ>
 struct IdxCfg {
   static constexpr int N = NQ * kIdxHeads;                 // MMA N
-  static constexpr int QPW = (NQ == 4) ? 2 : 1;            // queries per epilogue warp
-  static constexpr int EPI_WARPS = 4 * NQ / QPW;           // 8 or 4
+  static constexpr int EPI_WARPS = 4 * NQ;                 // a query per group of 4 lane-quarter warps
   static constexpr int EPI_THREADS = EPI_WARPS * 32;
+  static constexpr int GROUP_THREADS = 128;                // the threads of one query
   static constexpr int PRODUCER_WARP = EPI_WARPS;
   static constexpr int MMA_WARP = EPI_WARPS + 1;
   static constexpr int THREADS = (EPI_WARPS + 2) * 32;
@@ -51,7 +51,7 @@ struct IdxCfg {
   static constexpr int Q_BYTES = NQ * kIdxHeads * kIdxDim;
   static constexpr int K_BYTES = kKeyTile * kIdxDim;       // 16 KB
   static constexpr int TMEM_COLS = 2 * N;                  // two accumulators
-  static constexpr int MAXPER = kCand / EPI_THREADS;
+  static constexpr int MAXPER = kCand / GROUP_THREADS;
   // shared-memory layout (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
@@ -59,12 +59,13 @@ struct IdxCfg {
   static constexpr int OFF_POS = OFF_KEYS + NQ * kCand * 4;
   static constexpr int OFF_W = OFF_POS + NQ * kCand * 4;
   static constexpr int OFF_SEL = OFF_W + NQ * kIdxHeads * 4;
-  static constexpr int OFF_QST = OFF_SEL + static_cast<int>(sizeof(SelectScratch));
-  static constexpr int OFF_BAR = (OFF_QST + 3 * 4 * NQ + 8 + 16 + 7) & ~7;
+  static constexpr int OFF_QST = OFF_SEL + NQ * static_cast<int>(sizeof(SelectScratch));
+  static constexpr int OFF_BAR = (OFF_QST + 5 * 4 * NQ + 16 + 7) & ~7;
   static constexpr int NUM_BARS = 2 * STAGES + 2 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
-  static_assert(kCand % EPI_THREADS == 0, "candidate buffer must split evenly");
+  static_assert(kCand % GROUP_THREADS == 0, "candidate buffer must split evenly");
+  static_assert(THREADS <= 1024 && NQ <= 4, "block shape");
   static_assert(Q_BYTES % 1024 == 0 && K_BYTES % 1024 == 0, "swizzle atoms");
 };
 
@@ -262,22 +263,28 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     }
   } else {
     // ------------------------------------------------------------- epilogue warps
-    // Named barriers (bar.sync) cannot time out, so every epilogue warp must take the same
-    // path through them: mbarrier waits are done by lane 0 and broadcast, and the decision
-    // to stop after an abort is a snapshot taken by one thread between two barriers.
-    const uint32_t etid = threadIdx.x;                   // 0 .. EPI_THREADS-1
+    // Warps 4q .. 4q+3 own query q of the block, one TMEM lane quarter (32 keys) each; the
+    // four run as a group with their own named barrier (1 + q), candidate buffer and select
+    // scratch, so queries never wait for one another except through the shared accumulator.
+    // Named barriers (bar.sync) cannot time out, so every warp of a group takes the same path
+    // through them: mbarrier waits are done by lane 0 and broadcast, and the decision to stop
+    // after an abort is a snapshot taken by one thread of the group between two barriers.
+    const uint32_t q = warp >> 2;
     const uint32_t quarter = warp & 3u;
-    const uint32_t qset = warp >> 2;                     // which QPW queries of the block
+    const uint32_t gtid = threadIdx.x & (C::GROUP_THREADS - 1);
+    const uint32_t bar_id = 1u + q;
     const uint32_t lane_base = (quarter * 32u) << 16;
-    volatile uint32_t* snap = q_strict + NQ;             // two parity slots
+    SelectScratch* gsel = sel + q;
+    volatile uint32_t* snap = q_strict + NQ + 2 * q;     // two parity slots per group
+    uint32_t* cq_keys = cand_keys + q * kCand;
+    int32_t* cq_pos = cand_pos + q * kCand;
     uint32_t g = 0, nsync = 0;
-    // One barrier per step: thread 0 publishes the abort flag as it sees it into a parity
-    // slot before the barrier and everyone reads that slot after it. An abort raised while
-    // the slot was written is seen one step later, by all warps alike. A slot is rewritten
-    // two steps later, after every thread has read it.
+    // One barrier per step: thread 0 of the group publishes the abort flag as it sees it into
+    // a parity slot before the barrier and the group reads that slot after it. A slot is
+    // rewritten two steps later, after every thread of the group has read it.
     auto uniform_stop = [&]() -> bool {
-      if (etid == 0) snap[nsync & 1u] = (*abort_flag != 0) ? 1u : 0u;
-      named_barrier(1, C::EPI_THREADS);
+      if (gtid == 0) snap[nsync & 1u] = (*abort_flag != 0) ? 1u : 0u;
+      named_barrier(bar_id, C::GROUP_THREADS);
       return snap[(nsync++) & 1u] != 0;
     };
     bool stop = false;
@@ -285,138 +292,130 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       const int32_t u = item_of(r, cta, G);
       if (u >= p.n_items) break;
       const Item it = make_item<NQ>(p, u);
-      // per-query setup
-      for (uint32_t x = etid; x < NQ * kIdxHeads; x += C::EPI_THREADS) {
-        const int32_t i = it.i0 + static_cast<int32_t>(x / kIdxHeads);
+      const int32_t i = it.i0 + static_cast<int32_t>(q);
+      const bool q_valid = NQ == 1 || i < p.n_q;
+      // per-query setup: head weights with the query's scale folded in
+      if (gtid < static_cast<uint32_t>(kIdxHeads)) {
         float v = 0.f;
-        if (i < p.n_q) {
+        if (q_valid) {
           const size_t qt = static_cast<size_t>(it.b) * p.n_q + i;
-          v = __bfloat162float(p.w[qt * kIdxHeads + (x % kIdxHeads)]) * __ldg(p.q_scale + qt);
+          v = __bfloat162float(p.w[qt * kIdxHeads + gtid]) * __ldg(p.q_scale + qt);
         }
-        wq[x] = v;
+        wq[q * kIdxHeads + gtid] = v;
       }
-      if (etid < NQ) {
-        q_count[etid] = 0;
-        q_thr[etid] = 0;
-        q_strict[etid] = 0;
+      if (gtid == 0) {
+        q_count[q] = 0;
+        q_thr[q] = 0;
+        q_strict[q] = 0;
       }
-      named_barrier(1, C::EPI_THREADS);
-      int32_t qpos[C::QPW];
-#pragma unroll
-      for (int j = 0; j < C::QPW; ++j) {
-        const int32_t i = it.i0 + static_cast<int32_t>(qset * C::QPW + j);
-        qpos[j] = (i < p.n_q) ? it.len - p.n_q + i : -1;
-      }
+      named_barrier(bar_id, C::GROUP_THREADS);
+      const int32_t qpos = q_valid ? it.len - p.n_q + i : -1;
+      const float4* w4 = reinterpret_cast<const float4*>(wq + q * kIdxHeads);
+      const float* ks_row = p.k_scale + static_cast<size_t>(it.b) * p.max_len;
+      const int32_t s_lane = it.s_begin + static_cast<int32_t>(quarter * 32 + lane);
+      // the key scale of the next tile is loaded one tile ahead
+      auto key_scale = [&](int32_t t) -> float {
+        const int32_t s = s_lane + t * kKeyTile;
+        return (t < it.ntiles && s < it.s_end) ? __ldg(ks_row + s) : 0.f;
+      };
+      float ks_next = key_scale(0);
       for (int32_t t = 0; t < it.ntiles; ++t, ++g) {
         const uint32_t buf = g & 1u, acc_ph = (g >> 1) & 1u;
-        const int32_t s = it.s_begin + t * kKeyTile + static_cast<int32_t>(quarter * 32 + lane);
+        const int32_t s = s_lane + t * kKeyTile;
         const bool in_range = s < it.s_end;
-        const float ks = in_range ? __ldg(p.k_scale + static_cast<size_t>(it.b) * p.max_len + s) : 0.f;
+        const float ks = ks_next;
+        ks_next = key_scale(t + 1);
         // lane 0 waits; the warp then runs the collective TMEM loads together
         uint32_t got = 1;
         if (lane == 0) got = wt.wait(acc_full(buf), acc_ph, 8) ? 1u : 0u;
         const bool ok = __shfl_sync(0xffffffffu, got, 0) != 0;
         if (ok) {
-          uint32_t x[C::QPW][64];
+          uint32_t x[64];
           tc_fence_after();
-#pragma unroll
-          for (int j = 0; j < C::QPW; ++j) {
-            const uint32_t col = buf * C::N + (qset * C::QPW + j) * kIdxHeads;
-            tmem_ld32(tmem + lane_base + col, *reinterpret_cast<uint32_t(*)[32]>(&x[j][0]));
-            tmem_ld32(tmem + lane_base + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[j][32]));
-          }
+          const uint32_t col = buf * C::N + q * kIdxHeads;
+          tmem_ld32(tmem + lane_base + col, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+          tmem_ld32(tmem + lane_base + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(acc_empty(buf));
+          // sum_j w'_j * ReLU(x_j): packed fp32x2 FMAs over 4 independent accumulator pairs
+          float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                           make_float2(0.f, 0.f)};
 #pragma unroll
-          for (int j = 0; j < C::QPW; ++j) {
-            const uint32_t q = qset * C::QPW + j;
-            // sum_j w'_j * ReLU(x_j): packed fp32x2 FMAs over 4 independent accumulator pairs
-            const float4* w4 = reinterpret_cast<const float4*>(wq + q * kIdxHeads);
-            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                             make_float2(0.f, 0.f)};
-#pragma unroll
-            for (int h = 0; h < kIdxHeads; h += 4) {
-              const float4 wv = w4[h / 4];
-              const float2 r01 = make_float2(fmaxf(__uint_as_float(x[j][h + 0]), 0.f),
-                                             fmaxf(__uint_as_float(x[j][h + 1]), 0.f));
-              const float2 r23 = make_float2(fmaxf(__uint_as_float(x[j][h + 2]), 0.f),
-                                             fmaxf(__uint_as_float(x[j][h + 3]), 0.f));
-              const int c = (h / 4) & 1;
-              acc[2 * c] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc[2 * c]);
-              acc[2 * c + 1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc[2 * c + 1]);
-            }
-            const float score =
-                (((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y))) *
-                ks;
-            const uint32_t key = score_key(score);
-            const bool valid = in_range && s <= qpos[j];
-            const uint32_t thr = q_thr[q];
-            const bool pass = valid && (key > thr || (key == thr && q_strict[q] == 0));
-            const uint32_t m = __ballot_sync(0xffffffffu, pass);
-            if (m) {
-              uint32_t base = 0;
-              if (lane == 0) base = atomicAdd(&q_count[q], __popc(m));
-              base = __shfl_sync(0xffffffffu, base, 0);
-              if (pass) {
-                const uint32_t at = base + __popc(m & ((1u << lane) - 1u));
-                cand_keys[q * kCand + at] = key;
-                cand_pos[q * kCand + at] = s;
-              }
+          for (int h = 0; h < kIdxHeads; h += 4) {
+            const float4 wv = w4[h / 4];
+            const float2 r01 = make_float2(fmaxf(__uint_as_float(x[h + 0]), 0.f), fmaxf(__uint_as_float(x[h + 1]), 0.f));
+            const float2 r23 = make_float2(fmaxf(__uint_as_float(x[h + 2]), 0.f), fmaxf(__uint_as_float(x[h + 3]), 0.f));
+            const int c = (h / 4) & 1;
+            acc[2 * c] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc[2 * c]);
+            acc[2 * c + 1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc[2 * c + 1]);
+          }
+          const float score =
+              (((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y))) * ks;
+          const uint32_t key = score_key(score);
+          const bool valid = in_range && s <= qpos;
+          const uint32_t thr = q_thr[q];
+          const bool pass = valid && (key > thr || (key == thr && q_strict[q] == 0));
+          const uint32_t m = __ballot_sync(0xffffffffu, pass);
+          if (m) {
+            uint32_t base = 0;
+            if (lane == 0) base = atomicAdd(&q_count[q], __popc(m));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (pass) {
+              const uint32_t at = base + __popc(m & ((1u << lane) - 1u));
+              cq_keys[at] = key;
+              cq_pos[at] = s;
             }
           }
         }
         if (uniform_stop()) { stop = true; break; }
-        for (int q = 0; q < NQ; ++q) {
-          const uint32_t n = q_count[q];
-          if (n > static_cast<uint32_t>(kCand - kKeyTile)) {
-            // cheap range-histogram shrink; the exact select only if it frees too little
-            uint32_t thr = 0;
-            const uint32_t m = shrink_candidates<C::EPI_THREADS, C::MAXPER>(
-                cand_keys + q * kCand, cand_pos + q * kCand, n, static_cast<uint32_t>(p.topk), sel, etid, 1, &thr);
-            if (m > static_cast<uint32_t>((kCand + p.topk) / 2)) {
-              const uint32_t vk = select_exact<C::EPI_THREADS, C::MAXPER>(
-                  cand_keys + q * kCand, cand_pos + q * kCand, m, static_cast<uint32_t>(p.topk), sel, etid, 1);
-              if (etid == 0) {
-                q_count[q] = p.topk;
-                q_thr[q] = vk;
-                q_strict[q] = 1;
-              }
-            } else if (etid == 0) {
-              q_count[q] = m;
-              q_thr[q] = thr;
-              q_strict[q] = 0;
+        const uint32_t n = q_count[q];
+        if (n > static_cast<uint32_t>(kCand - kKeyTile)) {
+          // cheap range-histogram shrink; the exact select only if it frees too little
+          uint32_t thr = 0;
+          const uint32_t m = shrink_candidates<C::GROUP_THREADS, C::MAXPER>(
+              cq_keys, cq_pos, n, static_cast<uint32_t>(p.topk), gsel, gtid, bar_id, &thr);
+          if (m > static_cast<uint32_t>((kCand + p.topk) / 2)) {
+            const uint32_t vk = select_exact<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, m,
+                                                                          static_cast<uint32_t>(p.topk), gsel, gtid,
+                                                                          bar_id);
+            if (gtid == 0) {
+              q_count[q] = p.topk;
+              q_thr[q] = vk;
+              q_strict[q] = 1;
             }
-            named_barrier(1, C::EPI_THREADS);
+          } else if (gtid == 0) {
+            q_count[q] = m;
+            q_thr[q] = thr;
+            q_strict[q] = 0;
           }
+          named_barrier(bar_id, C::GROUP_THREADS);
         }
       }
       if (stop) break;
-      // ---- finish the item: exact k, then write
-      for (int q = 0; q < NQ; ++q) {
-        const int32_t i = it.i0 + q;
-        if (NQ > 1 && i >= p.n_q) break;
+      // ---- finish the query: exact k, then write
+      if (q_valid) {
         uint32_t n = q_count[q];
         if (n > static_cast<uint32_t>(p.topk)) {
-          select_exact<C::EPI_THREADS, C::MAXPER>(cand_keys + q * kCand, cand_pos + q * kCand, n,
-                                                  static_cast<uint32_t>(p.topk), sel, etid, 1);
+          select_exact<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, n, static_cast<uint32_t>(p.topk), gsel, gtid,
+                                                    bar_id);
           n = p.topk;
         }
         if (NQ == 1) {
           const size_t slot = static_cast<size_t>(it.b) * p.n_chunks + (it.s_begin / kDecodeChunk);
-          for (uint32_t j = etid; j < n; j += C::EPI_THREADS) {
-            p.part_keys[slot * p.topk + j] = cand_keys[j];
-            p.part_pos[slot * p.topk + j] = cand_pos[j];
+          for (uint32_t j = gtid; j < n; j += C::GROUP_THREADS) {
+            p.part_keys[slot * p.topk + j] = cq_keys[j];
+            p.part_pos[slot * p.topk + j] = cq_pos[j];
           }
-          if (etid == 0) p.part_count[slot] = static_cast<int32_t>(n);
+          if (gtid == 0) p.part_count[slot] = static_cast<int32_t>(n);
         } else {
           int32_t* dst = p.out_idx + (static_cast<size_t>(it.b) * p.n_q + i) * p.topk;
-          for (uint32_t j = etid; j < static_cast<uint32_t>(p.topk); j += C::EPI_THREADS)
-            dst[j] = j < n ? cand_pos[q * kCand + j] : -1;
+          for (uint32_t j = gtid; j < static_cast<uint32_t>(p.topk); j += C::GROUP_THREADS)
+            dst[j] = j < n ? cq_pos[j] : -1;
         }
       }
-      named_barrier(1, C::EPI_THREADS);
+      named_barrier(bar_id, C::GROUP_THREADS);
     }
   }
   // ---- teardown: every role reaches here (all waits are bounded)
