@@ -35,12 +35,15 @@ namespace dsa {
 constexpr int kIdxHeads = 64;     // H_I (padded)
 constexpr int kIdxDim = 128;      // d_I (padded), one 128-byte row per head / key
 constexpr int kKeyTile = 128;     // keys per MMA tile (M)
-constexpr int kCand = 3072;       // candidate capacity per query
+constexpr int kCand = 3584;       // candidate capacity per query
 constexpr int kDecodeChunk = 8192;  // keys per decode work item
+constexpr int kSyncTiles = 2;       // key tiles between two capacity checks of a candidate buffer
 
 template <int NQ>
 struct IdxCfg {
-  static constexpr int N = NQ * kIdxHeads;                 // MMA N
+  static constexpr int N = NQ * kIdxHeads;                 // accumulator columns per tile
+  static constexpr int HALVES = (NQ == 4) ? 2 : 1;         // MMAs per tile (query pairs)
+  static constexpr int NH = N / HALVES;                    // MMA N
   static constexpr int EPI_WARPS = 4 * NQ;                 // a query per group of 4 lane-quarter warps
   static constexpr int EPI_THREADS = EPI_WARPS * 32;
   static constexpr int GROUP_THREADS = 128;                // the threads of one query
@@ -61,10 +64,11 @@ struct IdxCfg {
   static constexpr int OFF_SEL = OFF_W + NQ * kIdxHeads * 4;
   static constexpr int OFF_QST = OFF_SEL + NQ * static_cast<int>(sizeof(SelectScratch));
   static constexpr int OFF_BAR = (OFF_QST + 5 * 4 * NQ + 16 + 7) & ~7;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 + 4 + 1;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 + 8 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(kCand % GROUP_THREADS == 0, "candidate buffer must split evenly");
+  static_assert(kCand - kSyncTiles * kKeyTile >= 2048, "a checked buffer must hold the largest k");
   static_assert(THREADS <= 1024 && NQ <= 4, "block shape");
   static_assert(Q_BYTES % 1024 == 0 && K_BYTES % 1024 == 0, "swizzle atoms");
 };
@@ -155,9 +159,10 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
   auto k_empty = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
   const uint32_t q_full = bar0 + 8u * (2 * C::STAGES);
   const uint32_t q_empty = q_full + 8;
-  auto acc_full = [&](int b) { return q_full + 16 + 8u * b; };
-  auto acc_empty = [&](int b) { return q_full + 32 + 8u * b; };
-  const uint32_t mma_done = q_full + 48;
+  // accumulator buffer b, half h (queries 2h, 2h+1 of a 4-query block)
+  auto acc_full = [&](uint32_t b, uint32_t h) { return q_full + 16 + 8u * (2 * b + h); };
+  auto acc_empty = [&](uint32_t b, uint32_t h) { return q_full + 48 + 8u * (2 * b + h); };
+  const uint32_t mma_done = q_full + 80;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -169,10 +174,11 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(acc_full(b), 1);
-      mbar_init(acc_empty(b), C::EPI_WARPS);
-    }
+    for (uint32_t b = 0; b < 2; ++b)
+      for (uint32_t h = 0; h < static_cast<uint32_t>(C::HALVES); ++h) {
+        mbar_init(acc_full(b, h), 1);
+        mbar_init(acc_empty(b, h), C::EPI_WARPS / C::HALVES);
+      }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -227,7 +233,7 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc(0, 0, 0, 0, kKeyTile, C::N);
+      constexpr uint32_t idesc = make_idesc(0, 0, 0, 0, kKeyTile, C::NH);
       uint32_t stage = 0, phase = 0, qph = 0, g = 0;
       for (int32_t r = 0;; ++r) {
         const int32_t u = item_of(r, cta, G);
@@ -240,18 +246,24 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         for (int32_t t = 0; t < it.ntiles; ++t, ++g) {
           const uint32_t buf = g & 1u, acc_ph = (g >> 1) & 1u;
           if (!wt.wait(k_full(stage), phase, 5)) { ok = false; break; }
-          if (!wt.wait(acc_empty(buf), acc_ph ^ 1u, 6)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t a_base = sbase + C::OFF_K + stage * C::K_BYTES;
-          const uint32_t b_base = sbase + C::OFF_Q;
+          // one MMA group per query pair, each announced on its own, so the two epilogue
+          // halves run staggered by half a tile
 #pragma unroll
-          for (int kk = 0; kk < kIdxDim / 32; ++kk) {
-            const uint64_t ad = sw128_desc(a_base + kk * 32, 1, 1024);
-            const uint64_t bd = sw128_desc(b_base + kk * 32, 1, 1024);
-            mma_f8_ss(tmem + buf * C::N, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          for (uint32_t h = 0; h < static_cast<uint32_t>(C::HALVES); ++h) {
+            if (!wt.wait(acc_empty(buf, h), acc_ph ^ 1u, 6)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t b_base = sbase + C::OFF_Q + h * C::NH * kIdxDim;
+#pragma unroll
+            for (int kk = 0; kk < kIdxDim / 32; ++kk) {
+              const uint64_t ad = sw128_desc(a_base + kk * 32, 1, 1024);
+              const uint64_t bd = sw128_desc(b_base + kk * 32, 1, 1024);
+              mma_f8_ss(tmem + buf * C::N + h * C::NH, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(acc_full(buf, h));
           }
+          if (!ok) break;
           tc_commit(k_empty(stage));
-          tc_commit(acc_full(buf));
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
         tc_commit(q_empty);
@@ -270,6 +282,7 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     // through them: mbarrier waits are done by lane 0 and broadcast, and the decision to stop
     // after an abort is a snapshot taken by one thread of the group between two barriers.
     const uint32_t q = warp >> 2;
+    const uint32_t half = q / (NQ / C::HALVES);
     const uint32_t quarter = warp & 3u;
     const uint32_t gtid = threadIdx.x & (C::GROUP_THREADS - 1);
     const uint32_t bar_id = 1u + q;
@@ -313,10 +326,10 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       const float4* w4 = reinterpret_cast<const float4*>(wq + q * kIdxHeads);
       const float* ks_row = p.k_scale + static_cast<size_t>(it.b) * p.max_len;
       const int32_t s_lane = it.s_begin + static_cast<int32_t>(quarter * 32 + lane);
-      // the key scale of the next tile is loaded one tile ahead
+      // the key scale of the next tile is loaded one tile ahead (clamped address; the value
+      // of a key past the range is never used)
       auto key_scale = [&](int32_t t) -> float {
-        const int32_t s = s_lane + t * kKeyTile;
-        return (t < it.ntiles && s < it.s_end) ? __ldg(ks_row + s) : 0.f;
+        return __ldg(ks_row + min(s_lane + t * kKeyTile, it.s_end - 1));
       };
       float ks_next = key_scale(0);
       for (int32_t t = 0; t < it.ntiles; ++t, ++g) {
@@ -325,10 +338,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         const bool in_range = s < it.s_end;
         const float ks = ks_next;
         ks_next = key_scale(t + 1);
-        // lane 0 waits; the warp then runs the collective TMEM loads together
-        uint32_t got = 1;
-        if (lane == 0) got = wt.wait(acc_full(buf), acc_ph, 8) ? 1u : 0u;
-        const bool ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+        // every lane waits (no divergent branch); the warp then runs the collective TMEM loads
+        const bool ok = __all_sync(0xffffffffu, wt.wait(acc_full(buf, half), acc_ph, 8)) != 0;
         if (ok) {
           uint32_t x[64];
           tc_fence_after();
@@ -338,7 +349,7 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty(buf));
+          if (lane == 0) mbar_arrive(acc_empty(buf, half));
           // sum_j w'_j * ReLU(x_j): packed fp32x2 FMAs over 4 independent accumulator pairs
           float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                            make_float2(0.f, 0.f)};
@@ -369,14 +380,18 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
             }
           }
         }
+        // capacity check every kSyncTiles tiles: between two checks at most kSyncTiles * 128
+        // candidates arrive, and a check leaves at most kCand - kSyncTiles * 128
+        if (t % kSyncTiles != kSyncTiles - 1 && t + 1 != it.ntiles) continue;
         if (uniform_stop()) { stop = true; break; }
         const uint32_t n = q_count[q];
-        if (n > static_cast<uint32_t>(kCand - kKeyTile)) {
+        if (n > static_cast<uint32_t>(kCand - kSyncTiles * kKeyTile)) {
           // cheap range-histogram shrink; the exact select only if it frees too little
           uint32_t thr = 0;
           const uint32_t m = shrink_candidates<C::GROUP_THREADS, C::MAXPER>(
               cq_keys, cq_pos, n, static_cast<uint32_t>(p.topk), gsel, gtid, bar_id, &thr);
-          if (m > static_cast<uint32_t>((kCand + p.topk) / 2)) {
+          // the exact select when the shrink freed less than half of the usable space
+          if (m > static_cast<uint32_t>(kCand - kSyncTiles * kKeyTile + p.topk) / 2) {
             const uint32_t vk = select_exact<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, m,
                                                                           static_cast<uint32_t>(p.topk), gsel, gtid,
                                                                           bar_id);

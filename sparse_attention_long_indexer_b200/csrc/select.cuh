@@ -2,10 +2,9 @@
 //
 // Keys are order-preserving 32-bit images of fp32 scores (larger score <=> larger key);
 // ranking is by key descending, then by position ascending (equal scores go to the lower
-// position). `select_exact` keeps exactly k of n > k candidates in place: an 8-bit MSB-first
-// radix select finds the k-th key v, a second radix select over positions resolves the
-// items equal to v, and one pass compacts. All `T` threads of the calling group execute it
-// together; synchronisation uses named barrier `bar_id`.
+// position). `select_exact` keeps exactly k of n > k candidates in place: histogram passes
+// over a shrinking key range find the bin holding the k-th key (down to a single key value
+// if needed), passes over positions resolve the items equal to it, and one pass compacts.
 #pragma once
 #include <cstdint>
 
@@ -24,7 +23,9 @@ struct SelectScratch {
   uint32_t bin;     // chosen digit
   uint32_t above;   // items strictly above the chosen bin (among the active prefix)
   uint32_t out_count;
-  uint32_t pad;
+  uint32_t cnt;     // items in the chosen bin
+  uint32_t wlo[8];  // per-warp minima / maxima of a group reduction
+  uint32_t whi[8];
 };
 
 // Adds 1 to hist[bin] for every lane with `active`, one shared atomic per distinct bin in
@@ -69,163 +70,239 @@ __device__ __forceinline__ void scan_pick(SelectScratch* sc, uint32_t rem) {
   }
 }
 
-// Keeps exactly k of the n candidates (n > k). Returns the k-th key; afterwards only
-// candidates strictly better than (that key, any larger position) may be added.
-template <int T, int MAXPER>
-__device__ uint32_t select_exact(uint32_t* keys, int32_t* pos, uint32_t n, uint32_t k, SelectScratch* sc,
-                                 uint32_t tid, uint32_t bar_id) {
-  // ---- phase 1: the k-th largest key
-  uint32_t prefix = 0, mask = 0, rem = k, n_eq = 0;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (uint32_t i = tid; i < 256; i += T) sc->hist[i] = 0;
-    named_barrier(bar_id, T);
-    for (uint32_t i0 = 0; i0 < n; i0 += T) {      // uniform trip count: hist_add is warp-collective
-      const uint32_t i = i0 + tid;
-      const uint32_t key = i < n ? keys[i] : 0u;
-      hist_add(sc->hist, (key >> shift) & 255u, i < n && (key & mask) == prefix);
-    }
-    named_barrier(bar_id, T);
-    if (tid < 32) scan_pick<true>(sc, rem);
-    named_barrier(bar_id, T);
-    uint32_t bin = sc->bin;
-    rem -= sc->above;
-    n_eq = sc->hist[bin];
-    prefix |= bin << shift;
-    mask |= 0xFFu << shift;
-    named_barrier(bar_id, T);
-  }
-  const uint32_t vk = prefix;
-  // ---- phase 2: among the n_eq items equal to vk keep the rem lowest positions
-  uint32_t plim = 0xFFFFFFFFu;
-  if (rem < n_eq) {
-    uint32_t pprefix = 0, pmask = 0, prem = rem;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (uint32_t i = tid; i < 256; i += T) sc->hist[i] = 0;
-      named_barrier(bar_id, T);
-      for (uint32_t i0 = 0; i0 < n; i0 += T) {
-        const uint32_t i = i0 + tid;
-        const uint32_t p = i < n ? static_cast<uint32_t>(pos[i]) : 0u;
-        hist_add(sc->hist, (p >> shift) & 255u, i < n && keys[i] == vk && (p & pmask) == pprefix);
-      }
-      named_barrier(bar_id, T);
-      if (tid < 32) scan_pick<false>(sc, prem);
-      named_barrier(bar_id, T);
-      prem -= sc->above;
-      pprefix |= sc->bin << shift;
-      pmask |= 0xFFu << shift;
-      named_barrier(bar_id, T);
-    }
-    plim = pprefix;
-  }
-  // ---- phase 3: compact in place (every item is read before any is written)
-  uint32_t rk[MAXPER];
-  int32_t rp[MAXPER];
-#pragma unroll
-  for (int j = 0; j < MAXPER; ++j) {
-    uint32_t i = tid + j * T;
-    rk[j] = 0;
-    rp[j] = -1;
-    if (i < n) {
-      rk[j] = keys[i];
-      rp[j] = pos[i];
-    }
-  }
-  if (tid == 0) sc->out_count = 0;
-  named_barrier(bar_id, T);
-  const uint32_t lane = threadIdx.x & 31;
-#pragma unroll
-  for (int j = 0; j < MAXPER; ++j) {
-    bool keep = (rp[j] >= 0) && (tid + j * T < n) &&
-                (rk[j] > vk || (rk[j] == vk && static_cast<uint32_t>(rp[j]) <= plim));
-    uint32_t m = __ballot_sync(0xffffffffu, keep);
-    if (m) {
-      uint32_t base = 0;
-      uint32_t leader = __ffs(m) - 1;
-      if (lane == leader) base = atomicAdd(&sc->out_count, __popc(m));
-      base = __shfl_sync(0xffffffffu, base, leader);
-      if (keep) {
-        uint32_t at = base + __popc(m & ((1u << lane) - 1u));
-        keys[at] = rk[j];
-        pos[at] = rp[j];
-      }
-    }
-  }
-  named_barrier(bar_id, T);
-  return vk;
-}
+// ------------------------------------------------------------------ register-resident selection
+// The candidates of a group are read once into registers (thread tid holds items tid + j*T);
+// histogram passes bin them over an adaptive key range with plain shared-memory atomics, and
+// the survivors are written back with one atomic per warp. All T threads of the group call
+// these together; synchronisation uses named barrier `bar_id`.
 
-// Cheap shrink used while streaming: keeps every candidate whose key is at least the lower
-// edge of the histogram bin holding the k-th largest key, bins splitting the current key
-// range [min, max] into 256 equal intervals. At least k candidates stay (typically k plus a
-// few), and everything dropped is strictly below k kept ones, so the returned threshold is
-// non-strict: later candidates equal to it must still be admitted. Returns the new count;
-// `*thr_out` receives the threshold.
 template <int T, int MAXPER>
-__device__ uint32_t shrink_candidates(uint32_t* keys, int32_t* pos, uint32_t n, uint32_t k, SelectScratch* sc,
-                                      uint32_t tid, uint32_t bar_id, uint32_t* thr_out) {
-  const uint32_t lane = threadIdx.x & 31;
-  uint32_t rk[MAXPER];
-  int32_t rp[MAXPER];
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+__device__ __forceinline__ void load_candidates(const uint32_t* keys, const int32_t* pos, uint32_t n, uint32_t tid,
+                                                uint32_t (&rk)[MAXPER], int32_t (&rp)[MAXPER]) {
 #pragma unroll
   for (int j = 0; j < MAXPER; ++j) {
     const uint32_t i = tid + j * T;
-    rk[j] = 0;
-    rp[j] = -1;
-    if (i < n) {
-      rk[j] = keys[i];
-      rp[j] = pos[i];
-      lo = min(lo, rk[j]);
-      hi = max(hi, rk[j]);
-    }
+    rk[j] = i < n ? keys[i] : 0u;
+    rp[j] = i < n ? pos[i] : -1;
   }
+}
+
+// Upper edge of the bin starting at b of width 2^shift, clamped to hi.
+__device__ __forceinline__ uint32_t bin_end(uint32_t b, uint32_t shift, uint32_t hi) {
+  const uint64_t e = static_cast<uint64_t>(b) + ((1ull << shift) - 1ull);
+  return e < hi ? static_cast<uint32_t>(e) : hi;
+}
+
+// Smallest shift that brings a value range below 256 bins.
+__device__ __forceinline__ uint32_t bin_shift(uint32_t range) { return range < 256u ? 0u : (32u - __clz(range)) - 8u; }
+
+// Group-wide min / max of v(j) over the items with act(j).
+template <int T, int MAXPER, typename Act, typename Val>
+__device__ __forceinline__ void group_minmax(Act act, Val v, SelectScratch* sc, uint32_t tid, uint32_t bar_id,
+                                             uint32_t& lo, uint32_t& hi) {
+  lo = 0xFFFFFFFFu;
+  hi = 0u;
+#pragma unroll
+  for (int j = 0; j < MAXPER; ++j)
+    if (act(j)) {
+      lo = min(lo, v(j));
+      hi = max(hi, v(j));
+    }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
     hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
   }
-  for (uint32_t i = tid; i < 256; i += T) sc->hist[i] = 0;
-  if (tid == 0) {
-    sc->bin = 0xFFFFFFFFu;   // running min
-    sc->above = 0u;          // running max
+  if ((threadIdx.x & 31) == 0) {
+    sc->wlo[tid >> 5] = lo;
+    sc->whi[tid >> 5] = hi;
   }
   named_barrier(bar_id, T);
-  if (lane == 0) {
-    atomicMin(&sc->bin, lo);
-    atomicMax(&sc->above, hi);
+#pragma unroll
+  for (int w = 0; w < T / 32; ++w) {
+    lo = min(lo, sc->wlo[w]);
+    hi = max(hi, sc->whi[w]);
   }
-  named_barrier(bar_id, T);
-  lo = sc->bin;
-  hi = sc->above;
-  const uint32_t range = hi - lo;
-  const uint32_t shift = range < 256u ? 0u : (32u - __clz(range)) - 8u;
+}
+
+// Warp 0 scans hist (descending or ascending bins) for the bin where the running count
+// first reaches `rem`; publishes the bin, the count before it and its own count.
+template <bool kDescending>
+__device__ __forceinline__ void scan_bins(SelectScratch* sc, uint32_t rem) {
+  const uint32_t lane = threadIdx.x & 31;
+  uint32_t loc[8];
+  uint32_t sum = 0;
 #pragma unroll
-  for (int j = 0; j < MAXPER; ++j) hist_add(sc->hist, (rk[j] - lo) >> shift, rp[j] >= 0);
-  named_barrier(bar_id, T);
-  if (tid < 32) scan_pick<true>(sc, k);
-  named_barrier(bar_id, T);
-  const uint32_t thr = lo + (sc->bin << shift);
-  if (tid == 0) sc->out_count = 0;
-  named_barrier(bar_id, T);
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t bin = kDescending ? (255u - 8u * lane - i) : (8u * lane + i);
+    loc[i] = sc->hist[bin];
+    sum += loc[i];
+  }
+  uint32_t incl = sum;
 #pragma unroll
-  for (int j = 0; j < MAXPER; ++j) {
-    const bool keep = rp[j] >= 0 && rk[j] >= thr;
-    const uint32_t m = __ballot_sync(0xffffffffu, keep);
-    if (m) {
-      uint32_t base = 0;
-      const uint32_t leader = __ffs(m) - 1;
-      if (lane == leader) base = atomicAdd(&sc->out_count, __popc(m));
-      base = __shfl_sync(0xffffffffu, base, leader);
-      if (keep) {
-        const uint32_t at = base + __popc(m & ((1u << lane) - 1u));
-        keys[at] = rk[j];
-        pos[at] = rp[j];
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= static_cast<uint32_t>(o)) incl += v;
+  }
+  uint32_t excl = incl - sum;
+  if (excl < rem && rem <= incl) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (excl + loc[i] >= rem) {
+        sc->bin = kDescending ? (255u - 8u * lane - i) : (8u * lane + i);
+        sc->above = excl;
+        sc->cnt = loc[i];
+        break;
       }
+      excl += loc[i];
     }
   }
+}
+
+// One histogram pass over the items with act(j), bin b(j) < 256.
+template <bool kDescending, int T, int MAXPER, typename Act, typename Bin>
+__device__ __forceinline__ void hist_pass(Act act, Bin b, uint32_t rem, SelectScratch* sc, uint32_t tid,
+                                          uint32_t bar_id, uint32_t& bin, uint32_t& above, uint32_t& cnt) {
+  for (uint32_t i = tid; i < 256; i += T) sc->hist[i] = 0;
   named_barrier(bar_id, T);
+#pragma unroll
+  for (int j = 0; j < MAXPER; ++j)
+    if (act(j)) atomicAdd(&sc->hist[b(j)], 1u);
+  named_barrier(bar_id, T);
+  if (tid < 32) scan_bins<kDescending>(sc, rem);
+  named_barrier(bar_id, T);
+  bin = sc->bin;
+  above = sc->above;
+  cnt = sc->cnt;
+}
+
+// Writes the kept register items to the front of keys/pos (any order), one atomic per warp.
+// Every thread must have loaded its items before the group's last barrier.
+template <int T, int MAXPER, typename Keep>
+__device__ __forceinline__ void compact_candidates(uint32_t* keys, int32_t* pos, const uint32_t (&rk)[MAXPER],
+                                                   const int32_t (&rp)[MAXPER], Keep keep, SelectScratch* sc,
+                                                   uint32_t bar_id) {
+  static_assert(MAXPER <= 32, "keep mask");
+  const uint32_t lane = threadIdx.x & 31;
+  uint32_t mask = 0, c = 0;
+#pragma unroll
+  for (int j = 0; j < MAXPER; ++j)
+    if (rp[j] >= 0 && keep(rk[j], rp[j])) {
+      mask |= 1u << j;
+      ++c;
+    }
+  uint32_t incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= static_cast<uint32_t>(o)) incl += v;
+  }
+  uint32_t base = 0;
+  if (lane == 31) base = atomicAdd(&sc->out_count, incl);
+  base = __shfl_sync(0xffffffffu, base, 31);
+  uint32_t at = base + incl - c;
+#pragma unroll
+  for (int j = 0; j < MAXPER; ++j)
+    if (mask & (1u << j)) {
+      keys[at] = rk[j];
+      pos[at] = rp[j];
+      ++at;
+    }
+  named_barrier(bar_id, T);
+}
+
+// Keeps exactly k of the n candidates (n > k): the k largest keys, equal keys ranked by the
+// lower position. Returns a threshold key t such that any later candidate with a key <= t
+// (and, being later, a larger position) cannot enter the top k.
+template <int T, int MAXPER>
+__device__ uint32_t select_exact(uint32_t* keys, int32_t* pos, uint32_t n, uint32_t k, SelectScratch* sc,
+                                 uint32_t tid, uint32_t bar_id) {
+  uint32_t rk[MAXPER];
+  int32_t rp[MAXPER];
+  load_candidates<T, MAXPER>(keys, pos, n, tid, rk, rp);
+  if (tid == 0) sc->out_count = 0;
+  uint32_t lo, hi;
+  group_minmax<T, MAXPER>([&](int j) { return rp[j] >= 0; }, [&](int j) { return rk[j]; }, sc, tid, bar_id, lo, hi);
+  // ---- key passes: narrow the active range to the bin holding the k-th largest key
+  uint32_t rem = k, shift = bin_shift(hi - lo), a_lo = lo, a_hi = hi;
+  uint32_t thr = 0, vk = 0;
+  bool ties = false;
+  while (true) {
+    uint32_t bin, above, cnt;
+    hist_pass<true, T, MAXPER>([&](int j) { return rp[j] >= 0 && rk[j] >= a_lo && rk[j] <= a_hi; },
+                               [&](int j) { return (rk[j] - a_lo) >> shift; }, rem, sc, tid, bar_id, bin, above, cnt);
+    rem -= above;
+    const uint32_t blo = a_lo + (bin << shift);
+    if (cnt == rem) {                 // the whole bin is in: keys >= blo are exactly the k
+      thr = blo;
+      break;
+    }
+    if (shift == 0) {                 // a single key value, more items than places: ties
+      vk = blo;
+      ties = true;
+      break;
+    }
+    a_hi = bin_end(blo, shift, a_hi);
+    a_lo = blo;
+    shift = shift > 8u ? shift - 8u : 0u;
+  }
+  if (!ties) {
+    compact_candidates<T, MAXPER>(keys, pos, rk, rp, [&](uint32_t key, int32_t) { return key >= thr; }, sc, bar_id);
+    return thr;
+  }
+  // ---- position passes among the items equal to vk: keep the rem lowest positions
+  uint32_t plo, phi;
+  group_minmax<T, MAXPER>([&](int j) { return rp[j] >= 0 && rk[j] == vk; },
+                          [&](int j) { return static_cast<uint32_t>(rp[j]); }, sc, tid, bar_id, plo, phi);
+  uint32_t pshift = bin_shift(phi - plo), p_lo = plo, p_hi = phi, plim = phi;
+  while (true) {
+    uint32_t bin, below, cnt;
+    hist_pass<false, T, MAXPER>(
+        [&](int j) {
+          const uint32_t pu = static_cast<uint32_t>(rp[j]);
+          return rp[j] >= 0 && rk[j] == vk && pu >= p_lo && pu <= p_hi;
+        },
+        [&](int j) { return (static_cast<uint32_t>(rp[j]) - p_lo) >> pshift; }, rem, sc, tid, bar_id, bin, below, cnt);
+    rem -= below;
+    const uint32_t pb = p_lo + (bin << pshift);
+    const uint32_t pe = bin_end(pb, pshift, p_hi);
+    if (cnt == rem || pshift == 0) {  // positions are distinct: a one-position bin holds one item
+      plim = pe;
+      break;
+    }
+    p_lo = pb;
+    p_hi = pe;
+    pshift = pshift > 8u ? pshift - 8u : 0u;
+  }
+  compact_candidates<T, MAXPER>(
+      keys, pos, rk, rp,
+      [&](uint32_t key, int32_t ps) { return key > vk || (key == vk && static_cast<uint32_t>(ps) <= plim); }, sc,
+      bar_id);
+  return vk;
+}
+
+// Cheap shrink used while streaming: one histogram pass over the candidates' key range
+// [min, max] in 256 equal bins keeps every candidate at or above the lower edge of the bin
+// holding the k-th largest key. At least k candidates stay, and everything dropped is below
+// k kept ones, so the returned threshold is non-strict: later candidates equal to it must
+// still be admitted. Returns the new count; `*thr_out` receives the threshold.
+template <int T, int MAXPER>
+__device__ uint32_t shrink_candidates(uint32_t* keys, int32_t* pos, uint32_t n, uint32_t k, SelectScratch* sc,
+                                      uint32_t tid, uint32_t bar_id, uint32_t* thr_out) {
+  uint32_t rk[MAXPER];
+  int32_t rp[MAXPER];
+  load_candidates<T, MAXPER>(keys, pos, n, tid, rk, rp);
+  if (tid == 0) sc->out_count = 0;
+  uint32_t lo, hi;
+  group_minmax<T, MAXPER>([&](int j) { return rp[j] >= 0; }, [&](int j) { return rk[j]; }, sc, tid, bar_id, lo, hi);
+  const uint32_t shift = bin_shift(hi - lo);
+  uint32_t bin, above, cnt;
+  hist_pass<true, T, MAXPER>([&](int j) { return rp[j] >= 0; }, [&](int j) { return (rk[j] - lo) >> shift; }, k, sc,
+                             tid, bar_id, bin, above, cnt);
+  const uint32_t thr = lo + (bin << shift);
+  compact_candidates<T, MAXPER>(keys, pos, rk, rp, [&](uint32_t key, int32_t) { return key >= thr; }, sc, bar_id);
   *thr_out = thr;
-  return sc->out_count;
+  return above + cnt;
 }
 
 }  // namespace dsa
