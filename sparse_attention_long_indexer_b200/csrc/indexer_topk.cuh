@@ -341,26 +341,32 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         // every lane waits (no divergent branch); the warp then runs the collective TMEM loads
         const bool ok = __all_sync(0xffffffffu, wt.wait(acc_full(buf, half), acc_ph, 8)) != 0;
         if (ok) {
-          uint32_t x[64];
+          uint32_t x[32];
           tc_fence_after();
           const uint32_t col = buf * C::N + q * kIdxHeads;
-          tmem_ld32(tmem + lane_base + col, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-          tmem_ld32(tmem + lane_base + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty(buf, half));
-          // sum_j w'_j * ReLU(x_j): packed fp32x2 FMAs over 4 independent accumulator pairs
+          // sum_j w'_j * ReLU(x_j): packed fp32x2 FMAs over 4 independent accumulator pairs; the
+          // 64 head columns come in two loads of 32 (fewer live registers), and the accumulator
+          // is released after the second
           float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                            make_float2(0.f, 0.f)};
 #pragma unroll
-          for (int h = 0; h < kIdxHeads; h += 4) {
-            const float4 wv = w4[h / 4];
-            const float2 r01 = make_float2(fmaxf(__uint_as_float(x[h + 0]), 0.f), fmaxf(__uint_as_float(x[h + 1]), 0.f));
-            const float2 r23 = make_float2(fmaxf(__uint_as_float(x[h + 2]), 0.f), fmaxf(__uint_as_float(x[h + 3]), 0.f));
-            const int c = (h / 4) & 1;
-            acc[2 * c] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc[2 * c]);
-            acc[2 * c + 1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc[2 * c + 1]);
+          for (int part = 0; part < 2; ++part) {
+            tmem_ld32(tmem + lane_base + col + 32 * part, x);
+            tmem_wait_ld();
+            if (part == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(acc_empty(buf, half));
+            }
+#pragma unroll
+            for (int h = 0; h < 32; h += 4) {
+              const float4 wv = w4[(32 * part + h) / 4];
+              const float2 r01 = make_float2(fmaxf(__uint_as_float(x[h + 0]), 0.f), fmaxf(__uint_as_float(x[h + 1]), 0.f));
+              const float2 r23 = make_float2(fmaxf(__uint_as_float(x[h + 2]), 0.f), fmaxf(__uint_as_float(x[h + 3]), 0.f));
+              const int c = (h / 4) & 1;
+              acc[2 * c] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc[2 * c]);
+              acc[2 * c + 1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc[2 * c + 1]);
+            }
           }
           const float score =
               (((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y))) * ks;
