@@ -150,7 +150,8 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
   auto sb_full2 = [&](int s) { return B(19 + s); };
   auto vr_full2 = [&](int s) { return B(22 + s); };
   const uint32_t q_full2 = B(24);
-  auto s_empty2 = [&](int i) { return B(25 + i); };
+  // B(25), B(26): unused (a logits buffer is known free once the P of the block that used it
+  // is announced: the softmax reads the logits before it writes P)
   const uint32_t p_full2 = B(27);
   const uint32_t o_empty2 = B(28);
   const uint32_t mma_done = B(29);
@@ -167,7 +168,6 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
       // softmax warps + output-ring producer warps (+ the MMA thread in the even CTA)
       mbar_init(info_empty(i), C::SOFTMAX_WARPS + 2 + (leader ? 1 : 0));
       mbar_init(s_full(i), 1);
-      mbar_init(s_empty2(i), 2 * C::SOFTMAX_WARPS);
       mbar_init(vr_empty(i), 1);
       mbar_init(vr_full2(i), 2 * 2);
     }
@@ -407,7 +407,9 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         // logits of the next block into TMEM buffer sb&1 from the next logits stage
         auto do_s = [&]() -> bool {
           if (!wt.wait(sb_full2(sst), sph, 22)) return false;
-          if (!wt.wait(s_empty2(sb & 1u), ((sb >> 1) & 1u) ^ 1u, 23)) return false;
+          // the TMEM logits buffer sb&1 was last written by the logits MMA two blocks back;
+          // its softmax read it before announcing that block's P, which this thread has
+          // already waited for (program order: p_full of every earlier block precedes here)
           tc_fence_after();
           const uint32_t sbuf = sbase + C::OFF_SB + sst * C::SB_BYTES;
           const uint32_t d = tmem + C::COL_S + 32u * (sb & 1u);
@@ -518,7 +520,6 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(at_leader(s_empty2(sb & 1u)));
         ++sb;
         const int32_t nvalid = min(32, total - b * kBlk - 32 * static_cast<int32_t>(half));
         float z[32];
