@@ -59,8 +59,9 @@ struct AttnCfg {
   static constexpr int SOFTMAX_WARPS = 4;
   static constexpr int PRODUCER_WARPS = 4;               // 2 gather the logits ring, 2 the output ring
   static constexpr int GROUP_THREADS = 64;
-  static constexpr int MMA_WARP = SOFTMAX_WARPS + PRODUCER_WARPS;
-  static constexpr int THREADS = (MMA_WARP + 1) * 32;
+  static constexpr int MMA_WARP = SOFTMAX_WARPS + PRODUCER_WARPS;   // logits MMAs (and TMEM owner)
+  static constexpr int PV_WARP = MMA_WARP + 1;                       // output MMAs
+  static constexpr int THREADS = (PV_WARP + 1) * 32;
   // TMEM columns
   static constexpr uint32_t COL_O = 0, COL_S = 256, COL_Q = 320, TMEM_COLS = 512;
   // shared memory
@@ -150,8 +151,9 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
   auto sb_full2 = [&](int s) { return B(19 + s); };
   auto vr_full2 = [&](int s) { return B(22 + s); };
   const uint32_t q_full2 = B(24);
-  // B(25), B(26): unused (a logits buffer is known free once the P of the block that used it
-  // is announced: the softmax reads the logits before it writes P)
+  // logits buffer i free again: arrived by the output-MMA thread once it has seen the P of the
+  // block that used the buffer (the softmax reads the logits before it writes P)
+  auto s_free = [&](int i) { return B(25 + i); };
   const uint32_t p_full2 = B(27);
   const uint32_t o_empty2 = B(28);
   const uint32_t mma_done = B(29);
@@ -166,7 +168,8 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     for (int i = 0; i < 2; ++i) {
       mbar_init(info_full(i), 1);
       // softmax warps + output-ring producer warps (+ the MMA thread in the even CTA)
-      mbar_init(info_empty(i), C::SOFTMAX_WARPS + 2 + (leader ? 1 : 0));
+      mbar_init(info_empty(i), C::SOFTMAX_WARPS + 2 + (leader ? 2 : 0));
+      mbar_init(s_free(i), 1);
       mbar_init(s_full(i), 1);
       mbar_init(vr_empty(i), 1);
       mbar_init(vr_full2(i), 2 * 2);
@@ -184,7 +187,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     mbar_init(q_full2, 2 * (1 + C::PRODUCER_WARPS));
     mbar_init(p_full2, 2 * C::SOFTMAX_WARPS);
     mbar_init(o_empty2, 2 * C::SOFTMAX_WARPS);
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -384,9 +387,13 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
       }
     }
     cp_async_wait<0>();
-  } else if (warp == C::MMA_WARP) {
-    // ================================================================ MMA issuer (even CTA only)
+  } else if (warp == C::MMA_WARP || warp == C::PV_WARP) {
+    // ================================================================ MMA issuers (even CTA only)
+    // Two threads feed the one tensor pipe so that each one's waits overlap the other's MMAs:
+    // warp MMA_WARP issues the logits MMAs, warp PV_WARP the output MMAs. A tcgen05.commit
+    // tracks the MMAs of its own thread, so each thread commits only what it issued.
     if (leader && lane == 0) {
+      const bool logits = warp == C::MMA_WARP;
       constexpr uint32_t idesc_s = make_idesc(1, 1, 0, 0, 128, kBlk);
       constexpr uint32_t idesc_o = make_idesc(1, 1, 0, 1, 128, 256);
       const uint32_t peer_off = mapa(bar0, 1) - bar0;
@@ -403,63 +410,61 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         mbar_arrive(info_empty(slot));
         const int32_t n_blocks = (total + kBlk - 1) / kBlk;
         if (n_blocks == 0) continue;
-        if (!wt.wait(q_full2, qq & 1u, 21)) break;
-        // logits of the next block into TMEM buffer sb&1 from the next logits stage
-        auto do_s = [&]() -> bool {
-          if (!wt.wait(sb_full2(sst), sph, 22)) return false;
-          // the TMEM logits buffer sb&1 was last written by the logits MMA two blocks back;
-          // its softmax read it before announcing that block's P, which this thread has
-          // already waited for (program order: p_full of every earlier block precedes here)
-          tc_fence_after();
-          const uint32_t sbuf = sbase + C::OFF_SB + sst * C::SB_BYTES;
-          const uint32_t d = tmem + C::COL_S + 32u * (sb & 1u);
+        if (logits) {
+          if (!wt.wait(q_full2, qq & 1u, 21)) break;
+          for (int32_t b = 0; b < n_blocks; ++b) {
+            // logits of block sb into TMEM buffer sb&1 from the next logits stage; the buffer
+            // was last written two blocks back and is free once that block's P was seen
+            if (!wt.wait(sb_full2(sst), sph, 22)) { ok = false; break; }
+            if (!wt.wait(s_free(sb & 1u), ((sb >> 1) & 1u) ^ 1u, 23)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sbuf = sbase + C::OFF_SB + sst * C::SB_BYTES;
+            const uint32_t d = tmem + C::COL_S + 32u * (sb & 1u);
 #pragma unroll
-          for (int j = 0; j < C::Q_TMEM_DIMS / 16; ++j) {      // A from TMEM
-            const int dj = 16 * j;
-            mma2_ts(d, tmem + C::COL_Q + 8 * j, sw128_desc(sbuf + (dj >> 6) * C::SB_ATOM + (dj & 63) * 2, 1, 1024),
-                    idesc_s, j > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int j = C::Q_TMEM_DIMS / 16; j < kDqk / 16; ++j) {   // A from shared memory
-            const int dj = 16 * j, dq = dj - C::Q_TMEM_DIMS;
-            mma2_ss(d, sw128_desc(sbase + C::OFF_QS + (dq >> 6) * 8192 + (dq & 63) * 2, 1, 1024),
-                    sw128_desc(sbuf + (dj >> 6) * C::SB_ATOM + (dj & 63) * 2, 1, 1024), idesc_s, 1u);
-          }
-          commit_both(s_full(sb & 1u));
-          commit_both(sb_empty(sst));
-          ++sb;
-          if (++sst == C::SB_STAGES) { sst = 0; sph ^= 1u; }
-          return true;
-        };
-        if (!do_s()) break;
-        for (int32_t b = 0; b < n_blocks; ++b) {
-          if (b + 1 < n_blocks) {
-            if (!do_s()) { ok = false; break; }
-          } else {
-            commit_both(q_empty);                  // every logits MMA of the query is issued
-          }
-          if (!wt.wait(vr_full2(vst), vph, 26)) { ok = false; break; }
-          if (!wt.wait(p_full2, pb & 1u, 24)) { ok = false; break; }
-          if (b == 0 && !wt.wait(o_empty2, (qq & 1u) ^ 1u, 25)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t vr = sbase + C::OFF_VR + vst * C::VR_BYTES;
-          const uint32_t pbuf = sbase + C::OFF_P;
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-#pragma unroll
-            for (int kk = 0; kk < kBlk / 16; ++kk) {
-              mma2_ss(tmem + C::COL_O + 128 * i, sw128_desc(pbuf + kk * 32, 1, 1024),
-                      sw128_desc(vr + 2 * i * C::VR_ATOM + kk * 2048, C::VR_ATOM, 1024), idesc_o,
-                      (b > 0 || kk > 0) ? 1u : 0u);
+            for (int j = 0; j < C::Q_TMEM_DIMS / 16; ++j) {      // A from TMEM
+              const int dj = 16 * j;
+              mma2_ts(d, tmem + C::COL_Q + 8 * j, sw128_desc(sbuf + (dj >> 6) * C::SB_ATOM + (dj & 63) * 2, 1, 1024),
+                      idesc_s, j > 0 ? 1u : 0u);
             }
+#pragma unroll
+            for (int j = C::Q_TMEM_DIMS / 16; j < kDqk / 16; ++j) {   // A from shared memory
+              const int dj = 16 * j, dq = dj - C::Q_TMEM_DIMS;
+              mma2_ss(d, sw128_desc(sbase + C::OFF_QS + (dq >> 6) * 8192 + (dq & 63) * 2, 1, 1024),
+                      sw128_desc(sbuf + (dj >> 6) * C::SB_ATOM + (dj & 63) * 2, 1, 1024), idesc_s, 1u);
+            }
+            commit_both(s_full(sb & 1u));
+            commit_both(sb_empty(sst));
+            ++sb;
+            if (++sst == C::SB_STAGES) { sst = 0; sph ^= 1u; }
           }
-          commit_both(vr_empty(vst));
-          commit_both(p_empty);
-          ++pb;
-          if (++vst == C::VR_STAGES) { vst = 0; vph ^= 1u; }
+          if (!ok) break;
+          commit_both(q_empty);                      // every logits MMA of the query is issued
+        } else {
+          for (int32_t b = 0; b < n_blocks; ++b) {
+            if (!wt.wait(vr_full2(vst), vph, 26)) { ok = false; break; }
+            if (!wt.wait(p_full2, pb & 1u, 24)) { ok = false; break; }
+            mbar_arrive(s_free(pb & 1u));            // the softmax is done with logits buffer pb&1
+            if (b == 0 && !wt.wait(o_empty2, (qq & 1u) ^ 1u, 25)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t vr = sbase + C::OFF_VR + vst * C::VR_BYTES;
+            const uint32_t pbuf = sbase + C::OFF_P;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+#pragma unroll
+              for (int kk = 0; kk < kBlk / 16; ++kk) {
+                mma2_ss(tmem + C::COL_O + 128 * i, sw128_desc(pbuf + kk * 32, 1, 1024),
+                        sw128_desc(vr + 2 * i * C::VR_ATOM + kk * 2048, C::VR_ATOM, 1024), idesc_o,
+                        (b > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
+            commit_both(vr_empty(vst));
+            commit_both(p_empty);
+            ++pb;
+            if (++vst == C::VR_STAGES) { vst = 0; vph ^= 1u; }
+          }
+          if (!ok) break;
+          commit_both(o_full);
         }
-        if (!ok) break;
-        commit_both(o_full);
         ++qq;
       }
       tc_commit(mma_done);
