@@ -154,7 +154,8 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
   // logits buffer i free again: arrived by the output-MMA thread once it has seen the P of the
   // block that used the buffer (the softmax reads the logits before it writes P)
   auto s_free = [&](int i) { return B(25 + i); };
-  const uint32_t p_full2 = B(27);
+  const uint32_t p_full2 = B(27);                        // even CTA: its softmax warps + the relay
+  const uint32_t p_local = B(30);                        // odd CTA: its softmax warps (relayed)
   const uint32_t o_empty2 = B(28);
   const uint32_t mma_done = B(29);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -168,7 +169,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     for (int i = 0; i < 2; ++i) {
       mbar_init(info_full(i), 1);
       // softmax warps + output-ring producer warps (+ the MMA thread in the even CTA)
-      mbar_init(info_empty(i), C::SOFTMAX_WARPS + 2 + (leader ? 2 : 0));
+      mbar_init(info_empty(i), C::SOFTMAX_WARPS + 2 + (leader ? 2 : 1));
       mbar_init(s_free(i), 1);
       mbar_init(s_full(i), 1);
       mbar_init(vr_empty(i), 1);
@@ -185,7 +186,8 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     for (int w = 0; w < 2; ++w)
       for (int par = 0; par < 2; ++par) mbar_init(pair_bar(w, par), 2);
     mbar_init(q_full2, 2 * (1 + C::PRODUCER_WARPS));
-    mbar_init(p_full2, 2 * C::SOFTMAX_WARPS);
+    mbar_init(p_full2, C::SOFTMAX_WARPS + 1);
+    mbar_init(p_local, C::SOFTMAX_WARPS);
     mbar_init(o_empty2, 2 * C::SOFTMAX_WARPS);
     mbar_init(mma_done, 2);
     *abort_flag = 0;
@@ -469,6 +471,24 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
       }
       tc_commit(mma_done);
       attn_drain_wait(mma_done, 0, p.wait_budget_ns);
+    } else if (!leader && warp == C::MMA_WARP && lane == 0) {
+      // relay of the odd CTA: its softmax warps announce P locally (a CTA-scope arrive does not
+      // stall them); this thread observes that (acquire) and forwards one cluster-scope release
+      // arrive to the even CTA, which by cumulativity carries the observed P stores
+      uint32_t qn = 0, pb = 0;
+      for (int32_t qi = cid; qi < p.n_queries; qi += ncl, ++qn) {
+        const uint32_t slot = qn & 1u, iph = (qn >> 1) & 1u;
+        if (!wt.wait(info_full(slot), iph, 27)) break;
+        const int32_t total = info[slot];
+        mbar_arrive(info_empty(slot));
+        const int32_t n_blocks = (total + kBlk - 1) / kBlk;
+        bool ok = true;
+        for (int32_t b = 0; b < n_blocks; ++b, ++pb) {
+          if (!wt.wait(p_local, pb & 1u, 28)) { ok = false; break; }
+          mbar_arrive_cluster(at_leader(p_full2));
+        }
+        if (!ok) break;
+      }
     }
   } else {
     // ================================================================ softmax warps (TMEM lane = thread)
@@ -586,7 +606,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(at_leader(p_full2));
+        if (lane == 0) mbar_arrive(leader ? p_full2 : p_local);
         ++pb;
       }
       if (!ok) break;
