@@ -46,30 +46,33 @@ constexpr int kBlk = 64;                 // selected rows per block
 constexpr int kMaxTopk = 2048;
 
 struct AttnCfg {
-  static constexpr int SB_STAGES = 3;                    // own rows, all dims (logits operand)
+  static constexpr int SB_STAGES = 2;                    // own rows, all dims (logits operand)
   static constexpr int VR_STAGES = 2;                    // all rows, this CTA's output dims
   static constexpr int SB_ATOM = 32 * 128;               // 32 rows x 128 B
   static constexpr int SB_BYTES = 9 * SB_ATOM;           // own 32 rows x 576 dims
   static constexpr int VR_ATOM = kBlk * 128;             // 64 rows x 128 B
   static constexpr int VR_BYTES = 4 * VR_ATOM;           // 64 rows x this CTA's 256 output dims
-  static constexpr int Q_TMEM_DIMS = 384;                // dims 0..383 of q in TMEM, the rest in smem
+  static constexpr int Q_TMEM_DIMS = 320;                // dims 0..319 of q in TMEM, the rest in smem
   static constexpr int QS_ATOMS = (kDqk - Q_TMEM_DIMS) / 64;
   static constexpr int QS_BYTES = QS_ATOMS * 64 * 128;   // 64 heads x dims 384..575
   static constexpr int P_BYTES = 64 * 128;               // 64 heads x 64 rows bf16
+  static constexpr int P_BUFS = 2;                       // P of two consecutive blocks
+  static constexpr int S_BUFS = 3;                       // TMEM logits buffers
   static constexpr int SOFTMAX_WARPS = 4;
-  static constexpr int PRODUCER_WARPS = 4;               // 2 gather the logits ring, 2 the output ring
-  static constexpr int GROUP_THREADS = 64;
+  static constexpr int PRODUCER_WARPS = 8;               // 4 gather the logits ring, 4 the output ring
+  static constexpr int GROUP_WARPS = PRODUCER_WARPS / 2;
+  static constexpr int GROUP_THREADS = GROUP_WARPS * 32;
   static constexpr int MMA_WARP = SOFTMAX_WARPS + PRODUCER_WARPS;   // logits MMAs (and TMEM owner)
   static constexpr int PV_WARP = MMA_WARP + 1;                       // output MMAs
   static constexpr int THREADS = (PV_WARP + 1) * 32;
   // TMEM columns
-  static constexpr uint32_t COL_O = 0, COL_S = 256, COL_Q = 320, TMEM_COLS = 512;
+  static constexpr uint32_t COL_O = 0, COL_S = 256, COL_Q = COL_S + 32 * S_BUFS, TMEM_COLS = 512;
   // shared memory
   static constexpr int OFF_SB = 0;
   static constexpr int OFF_VR = OFF_SB + SB_STAGES * SB_BYTES;
   static constexpr int OFF_QS = OFF_VR + VR_STAGES * VR_BYTES;
   static constexpr int OFF_P = OFF_QS + QS_BYTES;
-  static constexpr int OFF_SEL = OFF_P + P_BYTES;                  // 2 x kMaxTopk indices
+  static constexpr int OFF_SEL = OFF_P + P_BUFS * P_BYTES;         // 2 x kMaxTopk indices
   static constexpr int OFF_XMAX = OFF_SEL + 2 * kMaxTopk * 4;      // 2 x 128 floats
   static constexpr int OFF_SCAN = OFF_XMAX + 2 * 128 * 4;
   static constexpr int OFF_INFO = OFF_SCAN + 64;
@@ -143,8 +146,8 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
   auto vr_empty = [&](int s) { return B(7 + s); };       // commit: output operand stage consumed
   const uint32_t q_tma = B(9);                           // this CTA's smem part of q landed (TMA)
   const uint32_t q_empty = B(10);                        // commit: all logits MMAs of a query done
-  auto s_full = [&](int i) { return B(11 + i); };        // commit: logits buffer i ready
-  const uint32_t p_empty = B(13);                        // commit: output MMA that read P done
+  auto s_full = [&](uint32_t i) { return B(31 + i); };   // commit: logits buffer i ready (3)
+  auto p_empty = [&](uint32_t j) { return B(34 + j); };  // commit: output MMA that read P buffer j done (2)
   const uint32_t o_full = B(14);                         // commit: all output MMAs of a query done
   auto pair_bar = [&](int w, int par) { return B(15 + 2 * w + par); };   // softmax warp pairs
   // barriers of the even CTA, arrived on by both CTAs
@@ -153,9 +156,11 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
   const uint32_t q_full2 = B(24);
   // logits buffer i free again: arrived by the output-MMA thread once it has seen the P of the
   // block that used the buffer (the softmax reads the logits before it writes P)
-  auto s_free = [&](int i) { return B(25 + i); };
-  const uint32_t p_full2 = B(27);                        // even CTA: its softmax warps + the relay
-  const uint32_t p_local = B(30);                        // odd CTA: its softmax warps (relayed)
+  auto s_free = [&](uint32_t i) { return B(36 + i); };
+  // P buffer j announced (one barrier per buffer: a warp may announce the next block before a
+  // slower one has announced this one)
+  auto p_full2 = [&](uint32_t j) { return j ? B(39) : B(27); };   // even CTA: its softmax warps + relay
+  auto p_local = [&](uint32_t j) { return j ? B(11) : B(30); };   // odd CTA: its softmax warps
   const uint32_t o_empty2 = B(28);
   const uint32_t mma_done = B(29);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -169,25 +174,29 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     for (int i = 0; i < 2; ++i) {
       mbar_init(info_full(i), 1);
       // softmax warps + output-ring producer warps (+ the MMA thread in the even CTA)
-      mbar_init(info_empty(i), C::SOFTMAX_WARPS + 2 + (leader ? 2 : 1));
-      mbar_init(s_free(i), 1);
-      mbar_init(s_full(i), 1);
+      mbar_init(info_empty(i), C::SOFTMAX_WARPS + C::GROUP_WARPS + (leader ? 2 : 1));
       mbar_init(vr_empty(i), 1);
-      mbar_init(vr_full2(i), 2 * 2);
+      mbar_init(vr_full2(i), 2 * C::GROUP_WARPS);
     }
     for (int i = 0; i < C::SB_STAGES; ++i) {
       mbar_init(sb_empty(i), 1);
-      mbar_init(sb_full2(i), 2 * 2);
+      mbar_init(sb_full2(i), 2 * C::GROUP_WARPS);
     }
     mbar_init(q_tma, 1);
     mbar_init(q_empty, 1);
-    mbar_init(p_empty, 1);
+    for (uint32_t i = 0; i < static_cast<uint32_t>(C::S_BUFS); ++i) {
+      mbar_init(s_full(i), 1);
+      mbar_init(s_free(i), 1);
+    }
+    for (uint32_t j = 0; j < static_cast<uint32_t>(C::P_BUFS); ++j) mbar_init(p_empty(j), 1);
     mbar_init(o_full, 1);
     for (int w = 0; w < 2; ++w)
       for (int par = 0; par < 2; ++par) mbar_init(pair_bar(w, par), 2);
-    mbar_init(q_full2, 2 * (1 + C::PRODUCER_WARPS));
-    mbar_init(p_full2, C::SOFTMAX_WARPS + 1);
-    mbar_init(p_local, C::SOFTMAX_WARPS);
+    mbar_init(q_full2, 2 * (1 + C::GROUP_WARPS));
+    for (uint32_t j = 0; j < 2; ++j) {
+      mbar_init(p_full2(j), C::SOFTMAX_WARPS + 1);
+      mbar_init(p_local(j), C::SOFTMAX_WARPS);
+    }
     mbar_init(o_empty2, 2 * C::SOFTMAX_WARPS);
     mbar_init(mma_done, 2);
     *abort_flag = 0;
@@ -213,17 +222,18 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
 
   if (warp >= C::SOFTMAX_WARPS && warp < C::MMA_WARP) {
     // ================================================================ producers
-    // Group A (warps 4,5; TMEM lanes 0..63): index compaction, the q operand (TMA part and
-    // TMEM lanes 0..63), and the logits ring (this CTA's 32 rows of each block, all dims).
-    // Group B (warps 6,7; TMEM lanes 64..127): the duplicate q lanes and the output ring
-    // (all 64 rows of each block, the 256 output dims this CTA supplies).
+    // Group A (warps 4..7, one per TMEM lane quarter): index compaction, the q operand (TMA
+    // part, and the TMEM part in both lane halves), and the logits ring (this CTA's 32 rows of
+    // each block, all dims). Group B (warps 8..11): the output ring (all 64 rows of each block,
+    // the 256 output dims this CTA supplies).
     // Each group waits for its own copies (cp.async.wait_group, one group behind) and
     // announces a stage to the even CTA per warp; the rings are independent, so a stage is
     // announced without waiting for the other ring (no cycle through the MMA order).
     const uint32_t ptid = threadIdx.x - C::SOFTMAX_WARPS * 32;
-    const uint32_t pw = ptid >> 5;                     // 0..3 = TMEM lane quarter
-    const bool group_a = pw < 2;
-    const uint32_t gtid = ptid & 63u;
+    const uint32_t pw = ptid >> 5;                     // producer warp 0..7
+    const bool group_a = pw < static_cast<uint32_t>(C::GROUP_WARPS);
+    const uint32_t gw = pw % C::GROUP_WARPS;           // warp in group = TMEM lane quarter (group A)
+    const uint32_t gtid = ptid % C::GROUP_THREADS;
     volatile int32_t* go = scan + 8;
     const int32_t per = (p.topk + C::GROUP_THREADS - 1) / C::GROUP_THREADS;
     uint32_t qn = 0, nsync = 0, qq = 0;
@@ -261,10 +271,15 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
           const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
           if (static_cast<int32_t>(lane) >= o) incl += v;
         }
-        if (lane == 31) scan[pw] = incl;
+        if (lane == 31) scan[gw] = incl;
         named_barrier(2, C::GROUP_THREADS);
-        int32_t base = incl - cnt + (pw == 1 ? scan[0] : 0);
-        total = scan[0] + scan[1];
+        int32_t base = incl - cnt;
+        total = 0;
+#pragma unroll
+        for (int w = 0; w < C::GROUP_WARPS; ++w) {
+          base += (w < static_cast<int>(gw)) ? scan[w] : 0;
+          total += scan[w];
+        }
         for (int32_t j = j0; j < j1; ++j) {
           const int32_t v = __ldg(row + j);
           if (v >= 0 && v < p.max_len) sel[base++] = v;
@@ -280,9 +295,11 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
       }
       const int32_t n_blocks = (total + kBlk - 1) / kBlk;
       if (n_blocks > 0 && ok) {
-        // ---- the q operand: dims 384..575 by TMA into shared memory (group A thread 0),
-        // dims 0..383 into TMEM lanes of this warp (both lane halves: the same 64 heads)
-        if (warp_wait(q_empty, (qq & 1u) ^ 1u, 12)) {
+        // ---- the q operand (group A): dims Q_TMEM_DIMS.. by TMA into shared memory (thread 0),
+        // dims 0..Q_TMEM_DIMS-1 into this warp's TMEM lane quarter (both lane halves hold the
+        // same 64 heads)
+        if (!group_a) {
+        } else if (warp_wait(q_empty, (qq & 1u) ^ 1u, 12)) {
           if (ptid == 0) {
             mbar_expect_tx(q_tma, C::QS_BYTES);
             for (int a = 0; a < C::QS_ATOMS; ++a)
@@ -290,7 +307,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
                           qi * kHeads + 64 * static_cast<int32_t>(rank), 0);
           }
           tc_fence_after();
-          const uint32_t hl = ptid & 63u;
+          const uint32_t hl = gtid & 63u;
           const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(qi) * kHeads + 64 * rank + hl) *
                                                              kDqk);
 #pragma unroll 1
@@ -301,7 +318,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
               const uint4 u = __ldg(qsrc + c * 4 + v);
               r[4 * v + 0] = u.x; r[4 * v + 1] = u.y; r[4 * v + 2] = u.z; r[4 * v + 3] = u.w;
             }
-            tmem_st16(tmem + ((pw * 32u) << 16) + C::COL_Q + 16 * c, r);
+            tmem_st16(tmem + ((gw * 32u) << 16) + C::COL_Q + 16 * c, r);
           }
           tmem_wait_st();
           tc_fence_before();
@@ -313,7 +330,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         }
         ++qq;
         // ---- the ring of this group. Thread (r0, cc) copies 16-byte chunk cc of every 128-byte
-        // segment of block rows r0, r0 + 8, ...: the row indices are read once per block and each
+        // segment of block rows r0, r0 + GROUP_THREADS/8, ...: the row indices are read once per block and each
         // copy is a constant offset from the row's base, so copies issue back to back.
         const __nv_bfloat16* kv_seq = p.kv + static_cast<size_t>(qi / p.n_q) * p.max_len * kDqk;
         const uint32_t cc = gtid & 7u, r0 = gtid >> 3;
@@ -339,37 +356,40 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
           if (!warp_wait(empty_bar, ph ^ 1u, 11)) { ok = false; break; }
           if (group_a) {
             const uint32_t dst0 = sbase + C::OFF_SB + st * C::SB_BYTES + sw128_offset(r0, cc);
-            int32_t rows[4];
+            constexpr int RS = C::GROUP_THREADS / 8;       // rows per pass
+            int32_t rows[32 / RS];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int32_t j = b * kBlk + own0 + static_cast<int32_t>(r0) + 8 * q;
+            for (int q = 0; q < 32 / RS; ++q) {
+              const int32_t j = b * kBlk + own0 + static_cast<int32_t>(r0) + RS * q;
               rows[q] = j < total ? sel[j] : -1;
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 32 / RS; ++q) {
               const bool v = rows[q] >= 0;
               const __nv_bfloat16* src = (v ? kv_seq + static_cast<size_t>(rows[q]) * kDqk : p.kv) + cc * 8;
               const uint32_t n = v ? 16u : 0u;
 #pragma unroll
-              for (int a = 0; a < 9; ++a) cp_async_16(dst0 + q * 1024 + a * C::SB_ATOM, src + a * 64, n);
+              for (int a = 0; a < 9; ++a) cp_async_16(dst0 + q * RS * 128 + a * C::SB_ATOM, src + a * 64, n);
             }
           } else {
             const uint32_t dst0 = sbase + C::OFF_VR + st * C::VR_BYTES + sw128_offset(r0, cc);
-            int32_t rows[8];
+            constexpr int RS = C::GROUP_THREADS / 8;       // rows per pass
+            int32_t rows[kBlk / RS];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const int32_t j = b * kBlk + static_cast<int32_t>(r0) + 8 * q;
+            for (int q = 0; q < kBlk / RS; ++q) {
+              const int32_t j = b * kBlk + static_cast<int32_t>(r0) + RS * q;
               rows[q] = j < total ? sel[j] : -1;
             }
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < kBlk / RS; ++q) {
               const bool v = rows[q] >= 0;
               const __nv_bfloat16* src = (v ? kv_seq + static_cast<size_t>(rows[q]) * kDqk : p.kv) + seg0 + cc * 8;
               const uint32_t n = v ? 16u : 0u;
-              cp_async_16(dst0 + q * 1024 + 0 * C::VR_ATOM, src + 0, n);
-              cp_async_16(dst0 + q * 1024 + 1 * C::VR_ATOM, src + 64, n);
-              cp_async_16(dst0 + q * 1024 + 2 * C::VR_ATOM, src + 256, n);
-              cp_async_16(dst0 + q * 1024 + 3 * C::VR_ATOM, src + 320, n);
+              const uint32_t d = dst0 + q * RS * 128;
+              cp_async_16(d + 0 * C::VR_ATOM, src + 0, n);
+              cp_async_16(d + 1 * C::VR_ATOM, src + 64, n);
+              cp_async_16(d + 2 * C::VR_ATOM, src + 256, n);
+              cp_async_16(d + 3 * C::VR_ATOM, src + 320, n);
             }
           }
           cp_async_commit();
@@ -403,7 +423,8 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         commit2(local_bar);
         commit2(local_bar + peer_off);
       };
-      uint32_t sst = 0, sph = 0, vst = 0, vph = 0, qn = 0, sb = 0, pb = 0, qq = 0;
+      uint32_t sst = 0, sph = 0, vst = 0, vph = 0, qn = 0, pb = 0, qq = 0;
+      uint32_t s_i = 0, s_u = 0;                         // logits buffer, and its use count
       bool ok = true;
       for (int32_t qi = cid; qi < p.n_queries && ok; qi += ncl, ++qn) {
         const uint32_t slot = qn & 1u, iph = (qn >> 1) & 1u;
@@ -415,13 +436,13 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         if (logits) {
           if (!wt.wait(q_full2, qq & 1u, 21)) break;
           for (int32_t b = 0; b < n_blocks; ++b) {
-            // logits of block sb into TMEM buffer sb&1 from the next logits stage; the buffer
-            // was last written two blocks back and is free once that block's P was seen
+            // logits of the next block into TMEM buffer s_i from the next logits stage; the
+            // buffer was last written three blocks back and is free once that block's P was seen
             if (!wt.wait(sb_full2(sst), sph, 22)) { ok = false; break; }
-            if (!wt.wait(s_free(sb & 1u), ((sb >> 1) & 1u) ^ 1u, 23)) { ok = false; break; }
+            if (!wt.wait(s_free(s_i), (s_u & 1u) ^ 1u, 23)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sbuf = sbase + C::OFF_SB + sst * C::SB_BYTES;
-            const uint32_t d = tmem + C::COL_S + 32u * (sb & 1u);
+            const uint32_t d = tmem + C::COL_S + 32u * s_i;
 #pragma unroll
             for (int j = 0; j < C::Q_TMEM_DIMS / 16; ++j) {      // A from TMEM
               const int dj = 16 * j;
@@ -434,9 +455,9 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
               mma2_ss(d, sw128_desc(sbase + C::OFF_QS + (dq >> 6) * 8192 + (dq & 63) * 2, 1, 1024),
                       sw128_desc(sbuf + (dj >> 6) * C::SB_ATOM + (dj & 63) * 2, 1, 1024), idesc_s, 1u);
             }
-            commit_both(s_full(sb & 1u));
+            commit_both(s_full(s_i));
             commit_both(sb_empty(sst));
-            ++sb;
+            if (++s_i == static_cast<uint32_t>(C::S_BUFS)) { s_i = 0; ++s_u; }
             if (++sst == C::SB_STAGES) { sst = 0; sph ^= 1u; }
           }
           if (!ok) break;
@@ -444,12 +465,12 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         } else {
           for (int32_t b = 0; b < n_blocks; ++b) {
             if (!wt.wait(vr_full2(vst), vph, 26)) { ok = false; break; }
-            if (!wt.wait(p_full2, pb & 1u, 24)) { ok = false; break; }
-            mbar_arrive(s_free(pb & 1u));            // the softmax is done with logits buffer pb&1
+            if (!wt.wait(p_full2(pb & 1u), (pb >> 1) & 1u, 24)) { ok = false; break; }
+            mbar_arrive(s_free(pb % C::S_BUFS));     // the softmax is done with that logits buffer
             if (b == 0 && !wt.wait(o_empty2, (qq & 1u) ^ 1u, 25)) { ok = false; break; }
             tc_fence_after();
             const uint32_t vr = sbase + C::OFF_VR + vst * C::VR_BYTES;
-            const uint32_t pbuf = sbase + C::OFF_P;
+            const uint32_t pbuf = sbase + C::OFF_P + (pb & 1u) * C::P_BYTES;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
 #pragma unroll
@@ -460,7 +481,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
               }
             }
             commit_both(vr_empty(vst));
-            commit_both(p_empty);
+            commit_both(p_empty(pb & 1u));
             ++pb;
             if (++vst == C::VR_STAGES) { vst = 0; vph ^= 1u; }
           }
@@ -484,8 +505,8 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         const int32_t n_blocks = (total + kBlk - 1) / kBlk;
         bool ok = true;
         for (int32_t b = 0; b < n_blocks; ++b, ++pb) {
-          if (!wt.wait(p_local, pb & 1u, 28)) { ok = false; break; }
-          mbar_arrive_cluster(at_leader(p_full2));
+          if (!wt.wait(p_local(pb & 1u), (pb >> 1) & 1u, 28)) { ok = false; break; }
+          mbar_arrive_cluster(at_leader(p_full2(pb & 1u)));
         }
         if (!ok) break;
       }
@@ -501,7 +522,8 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     const uint32_t lane_off = (warp * 32u) << 16;
     const uint32_t pairw = warp & 1u;                  // warps 0,2 -> pair 0; 1,3 -> pair 1
     const uint32_t partner = L ^ 64u;
-    uint32_t qn = 0, sb = 0, pb = 0, nx = 0, qd = 0;
+    uint32_t qn = 0, pb = 0, nx = 0, qd = 0;
+    uint32_t s_i = 0, s_u = 0;                         // logits buffer, and its use count
     bool ok = true;
     // one float from the partner lane (the other half of the same head)
     auto swap_partner = [&](float mine) -> float {
@@ -537,15 +559,15 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
       float m2 = -INFINITY, l = 0.f;
       for (int32_t b = 0; b < n_blocks && ok; ++b) {
         // ---- this lane's 32 logits
-        if (lane == 0) got = wt.wait(s_full(sb & 1u), (sb >> 1) & 1u, 32) ? 1u : 0u;
+        if (lane == 0) got = wt.wait(s_full(s_i), s_u & 1u, 32) ? 1u : 0u;
         if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[32];
-        tmem_ld32(tmem + lane_off + C::COL_S + 32u * (sb & 1u), sr);
+        tmem_ld32(tmem + lane_off + C::COL_S + 32u * s_i, sr);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        ++sb;
+        if (++s_i == static_cast<uint32_t>(C::S_BUFS)) { s_i = 0; ++s_u; }
         const int32_t nvalid = min(32, total - b * kBlk - 32 * static_cast<int32_t>(half));
         float z[32];
         float mb = -INFINITY;
@@ -573,13 +595,18 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
           pk[j] = *reinterpret_cast<const uint32_t*>(&pr);
         }
         l += lsum;
-        // ---- the P buffer is free, and O stable, once the previous output MMA has finished
-        if (pb >= 1) {
-          if (lane == 0) got = wt.wait(p_empty, (pb - 1) & 1u, 35) ? 1u : 0u;
+        // ---- P buffer pb&1 is free once the output MMA of block pb-2 has finished; a rescale of O
+        // needs the one of block pb-1 finished too (it also implies the earlier one)
+        const bool rescale = __any_sync(0xffffffffu, need) && b > 0;
+        if (rescale && pb >= 1) {
+          if (lane == 0) got = wt.wait(p_empty((pb - 1) & 1u), ((pb - 1) >> 1) & 1u, 35) ? 1u : 0u;
+          if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
+        } else if (pb >= 2) {
+          if (lane == 0) got = wt.wait(p_empty(pb & 1u), ((pb >> 1) & 1u) ^ 1u, 34) ? 1u : 0u;
           if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
         }
         // ---- rescale this lane's output columns if the running max moved
-        if (__any_sync(0xffffffffu, need) && b > 0) {
+        if (rescale) {
           tc_fence_after();
           const float a = need ? alpha : 1.0f;
 #pragma unroll 1
@@ -596,7 +623,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         }
         {
           // P row hl, columns 32*half .. +31 (64 B = 4 chunks of the 128-byte swizzled row)
-          const uint32_t prow = sbase + C::OFF_P;
+          const uint32_t prow = sbase + C::OFF_P + (pb & 1u) * C::P_BYTES;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(prow + sw128_offset(hl, 4 * half + c)),
@@ -606,7 +633,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(leader ? p_full2 : p_local);
+        if (lane == 0) mbar_arrive(leader ? p_full2(pb & 1u) : p_local(pb & 1u));
         ++pb;
       }
       if (!ok) break;
