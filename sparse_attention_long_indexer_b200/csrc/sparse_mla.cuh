@@ -9,28 +9,33 @@
 //
 // B200 design. The fp32 output accumulator of one query (128 heads x 512 dims) is 256 KB,
 // all of one SM's tensor memory, so each query runs on a pair of CTAs (a 2-CTA cluster) and
-// every product is a 2-SM tcgen05 MMA (cta_group::2) issued by one thread of the even CTA:
+// every product is a 2-SM tcgen05 MMA (cta_group::2) issued from the even CTA:
 //  * logits: M = 128 heads (CTA r supplies heads 64r..64r+63), N = 64 selected rows (CTA r
 //    supplies block rows 32r..32r+31), K = 576. The hardware shares the halves and each CTA
 //    receives the logits of its own 64 heads for all 64 rows, folded in TMEM as 128 lanes x
-//    32 columns (lane m: rows 0..31 of head m, lane 64+m: rows 32..63). Dims 0..287 of Q come
-//    from TMEM (A operand, duplicated over both lane halves), dims 288..575 from shared memory.
+//    32 columns (lane m: rows 0..31 of head m, lane 64+m: rows 32..63); three such buffers.
+//    Dims 0..319 of Q come from TMEM (A operand, duplicated over both lane halves), dims
+//    320..575 from shared memory.
 //  * output: M = 128 heads, N = 256 latent dims per instruction (two instructions), K = 64
-//    rows: A = P (bf16, this CTA's heads) in shared memory, B = the rows' latent dims with CTA
-//    r supplying dims 256i + 128r .. +127. Each CTA accumulates all 512 dims of its 64 heads
-//    (TMEM: 256 columns; lane m / 64+m hold the low / high 128 dims of each instruction).
-//  * per 64-row block, CTA r gathers its 32 rows completely (logits operand, a 3-stage ring
+//    rows: A = P (bf16, this CTA's heads, two buffers) in shared memory, B = the rows' latent
+//    dims with CTA r supplying dims 256i + 128r .. +127. Each CTA accumulates all 512 dims of
+//    its 64 heads (TMEM: 256 columns; lane m / 64+m hold the low / high 128 dims of each
+//    instruction).
+//  * per 64-row block, CTA r gathers its 32 rows completely (logits operand, a 2-stage ring
 //    freed by the logits MMA) and all 64 rows' dims it supplies to the output product (a
 //    2-stage ring freed by the output MMA), with 16-byte cp.async into 128-byte-swizzled
-//    stages; two producer warp pairs run the two rings independently.
+//    stages; two groups of four producer warps run the two rings independently.
 //  * softmax: one thread per TMEM lane holds half a row (32 logits); the two halves of a row
 //    exchange their maxima through shared memory; online softmax in the log2 domain, the
 //    output rescaled only when the running max grows by more than 8 (exact: the final
-//    normalisation uses the same max). The logits of block b+1 are computed while the
-//    softmax of block b runs (two TMEM logit buffers).
+//    normalisation uses the same max). P is announced with a CTA-scope arrive; the odd CTA's
+//    announcements reach the even CTA through one relay thread.
+//  * two issuing threads share the tensor pipe: one for the logits MMAs, one for the output
+//    MMAs; the output thread hands a logits buffer back once it has seen that block's P, so
+//    the logits -> softmax -> P -> logits loop spans three blocks.
 // Nothing crosses between the two CTAs except through the 2-SM MMAs themselves; the pair
 // synchronises through mbarriers of the even CTA (remote arrives) and commits that the MMA
-// thread addresses to both CTAs.
+// threads address to both CTAs.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
