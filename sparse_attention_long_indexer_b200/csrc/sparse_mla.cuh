@@ -51,18 +51,18 @@ constexpr int kBlk = 64;                 // selected rows per block
 constexpr int kMaxTopk = 2048;
 
 struct AttnCfg {
-  static constexpr int SB_STAGES = 2;                    // own rows, all dims (logits operand)
+  static constexpr int SB_STAGES = 3;                    // own rows, all dims (logits operand)
   static constexpr int VR_STAGES = 2;                    // all rows, this CTA's output dims
   static constexpr int SB_ATOM = 32 * 128;               // 32 rows x 128 B
   static constexpr int SB_BYTES = 9 * SB_ATOM;           // own 32 rows x 576 dims
   static constexpr int VR_ATOM = kBlk * 128;             // 64 rows x 128 B
   static constexpr int VR_BYTES = 4 * VR_ATOM;           // 64 rows x this CTA's 256 output dims
-  static constexpr int Q_TMEM_DIMS = 320;                // dims 0..319 of q in TMEM, the rest in smem
+  static constexpr int Q_TMEM_DIMS = 384;                // dims 0..383 of q in TMEM, the rest in smem
   static constexpr int QS_ATOMS = (kDqk - Q_TMEM_DIMS) / 64;
   static constexpr int QS_BYTES = QS_ATOMS * 64 * 128;   // 64 heads x dims 384..575
   static constexpr int P_BYTES = 64 * 128;               // 64 heads x 64 rows bf16
-  static constexpr int P_BUFS = 2;                       // P of two consecutive blocks
-  static constexpr int S_BUFS = 3;                       // TMEM logits buffers
+  static constexpr int P_BUFS = 1;                       // P of consecutive blocks (1 or 2)
+  static constexpr int S_BUFS = 2;                       // TMEM logits buffers
   static constexpr int SOFTMAX_WARPS = 4;
   static constexpr int PRODUCER_WARPS = 8;               // 4 gather the logits ring, 4 the output ring
   static constexpr int GROUP_WARPS = PRODUCER_WARPS / 2;
@@ -88,6 +88,7 @@ struct AttnCfg {
   static_assert(OFF_VR % 1024 == 0 && OFF_QS % 1024 == 0 && OFF_P % 1024 == 0, "swizzle atoms");
   static_assert(SB_BYTES % 1024 == 0 && Q_TMEM_DIMS / 2 + COL_Q <= TMEM_COLS, "layout");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(P_BUFS == 1 || P_BUFS == 2, "P buffers");
 };
 
 struct AttnParams {
@@ -165,6 +166,8 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
   // P buffer j announced (one barrier per buffer: a warp may announce the next block before a
   // slower one has announced this one)
   auto p_full2 = [&](uint32_t j) { return j ? B(39) : B(27); };   // even CTA: its softmax warps + relay
+  auto pbuf_of = [](uint32_t n) { return n % static_cast<uint32_t>(C::P_BUFS); };        // P buffer of block n
+  auto puse_of = [](uint32_t n) { return (n / static_cast<uint32_t>(C::P_BUFS)) & 1u; }; // parity of its use
   auto p_local = [&](uint32_t j) { return j ? B(11) : B(30); };   // odd CTA: its softmax warps
   const uint32_t o_empty2 = B(28);
   const uint32_t mma_done = B(29);
@@ -198,7 +201,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     for (int w = 0; w < 2; ++w)
       for (int par = 0; par < 2; ++par) mbar_init(pair_bar(w, par), 2);
     mbar_init(q_full2, 2 * (1 + C::GROUP_WARPS));
-    for (uint32_t j = 0; j < 2; ++j) {
+    for (uint32_t j = 0; j < static_cast<uint32_t>(C::P_BUFS); ++j) {
       mbar_init(p_full2(j), C::SOFTMAX_WARPS + 1);
       mbar_init(p_local(j), C::SOFTMAX_WARPS);
     }
@@ -470,12 +473,12 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         } else {
           for (int32_t b = 0; b < n_blocks; ++b) {
             if (!wt.wait(vr_full2(vst), vph, 26)) { ok = false; break; }
-            if (!wt.wait(p_full2(pb & 1u), (pb >> 1) & 1u, 24)) { ok = false; break; }
+            if (!wt.wait(p_full2(pbuf_of(pb)), puse_of(pb), 24)) { ok = false; break; }
             mbar_arrive(s_free(pb % C::S_BUFS));     // the softmax is done with that logits buffer
             if (b == 0 && !wt.wait(o_empty2, (qq & 1u) ^ 1u, 25)) { ok = false; break; }
             tc_fence_after();
             const uint32_t vr = sbase + C::OFF_VR + vst * C::VR_BYTES;
-            const uint32_t pbuf = sbase + C::OFF_P + (pb & 1u) * C::P_BYTES;
+            const uint32_t pbuf = sbase + C::OFF_P + pbuf_of(pb) * C::P_BYTES;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
 #pragma unroll
@@ -486,7 +489,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
               }
             }
             commit_both(vr_empty(vst));
-            commit_both(p_empty(pb & 1u));
+            commit_both(p_empty(pbuf_of(pb)));
             ++pb;
             if (++vst == C::VR_STAGES) { vst = 0; vph ^= 1u; }
           }
@@ -510,8 +513,8 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         const int32_t n_blocks = (total + kBlk - 1) / kBlk;
         bool ok = true;
         for (int32_t b = 0; b < n_blocks; ++b, ++pb) {
-          if (!wt.wait(p_local(pb & 1u), (pb >> 1) & 1u, 28)) { ok = false; break; }
-          mbar_arrive_cluster(at_leader(p_full2(pb & 1u)));
+          if (!wt.wait(p_local(pbuf_of(pb)), puse_of(pb), 28)) { ok = false; break; }
+          mbar_arrive_cluster(at_leader(p_full2(pbuf_of(pb))));
         }
         if (!ok) break;
       }
@@ -600,14 +603,14 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
           pk[j] = *reinterpret_cast<const uint32_t*>(&pr);
         }
         l += lsum;
-        // ---- P buffer pb&1 is free once the output MMA of block pb-2 has finished; a rescale of O
-        // needs the one of block pb-1 finished too (it also implies the earlier one)
+        // ---- the P buffer of block pb is free once the output MMA of block pb - P_BUFS has
+        // finished; a rescale of O needs the one of block pb-1 finished (it implies the earlier ones)
         const bool rescale = __any_sync(0xffffffffu, need) && b > 0;
         if (rescale && pb >= 1) {
-          if (lane == 0) got = wt.wait(p_empty((pb - 1) & 1u), ((pb - 1) >> 1) & 1u, 35) ? 1u : 0u;
+          if (lane == 0) got = wt.wait(p_empty(pbuf_of(pb - 1)), puse_of(pb - 1), 35) ? 1u : 0u;
           if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
-        } else if (pb >= 2) {
-          if (lane == 0) got = wt.wait(p_empty(pb & 1u), ((pb >> 1) & 1u) ^ 1u, 34) ? 1u : 0u;
+        } else if (pb >= static_cast<uint32_t>(C::P_BUFS)) {
+          if (lane == 0) got = wt.wait(p_empty(pbuf_of(pb)), puse_of(pb) ^ 1u, 34) ? 1u : 0u;
           if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
         }
         // ---- rescale this lane's output columns if the running max moved
@@ -628,7 +631,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         }
         {
           // P row hl, columns 32*half .. +31 (64 B = 4 chunks of the 128-byte swizzled row)
-          const uint32_t prow = sbase + C::OFF_P + (pb & 1u) * C::P_BYTES;
+          const uint32_t prow = sbase + C::OFF_P + pbuf_of(pb) * C::P_BYTES;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(prow + sw128_offset(hl, 4 * half + c)),
@@ -638,7 +641,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(leader ? p_full2(pb & 1u) : p_local(pb & 1u));
+        if (lane == 0) mbar_arrive(leader ? p_full2(pbuf_of(pb)) : p_local(pbuf_of(pb)));
         ++pb;
       }
       if (!ok) break;
