@@ -77,8 +77,9 @@ struct AttnCfg {
   static constexpr int OFF_VR = OFF_SB + SB_STAGES * SB_BYTES;
   static constexpr int OFF_QS = OFF_VR + VR_STAGES * VR_BYTES;
   static constexpr int OFF_P = OFF_QS + QS_BYTES;
-  static constexpr int OFF_SEL = OFF_P + P_BUFS * P_BYTES;         // 2 x kMaxTopk indices
-  static constexpr int OFF_XMAX = OFF_SEL + 2 * kMaxTopk * 4;      // 2 x 128 floats
+  static constexpr int SEL_BUFS = 2;                     // compacted index lists (1 or 2)
+  static constexpr int OFF_SEL = OFF_P + P_BUFS * P_BYTES;         // SEL_BUFS x kMaxTopk indices
+  static constexpr int OFF_XMAX = OFF_SEL + SEL_BUFS * kMaxTopk * 4;  // 2 x 128 floats
   static constexpr int OFF_SCAN = OFF_XMAX + 2 * 128 * 4;
   static constexpr int OFF_INFO = OFF_SCAN + 64;
   static constexpr int OFF_BAR = OFF_INFO + 16;
@@ -260,10 +261,13 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     };
     for (int32_t qi = cid; qi < p.n_queries; qi += ncl, ++qn) {
       const uint32_t slot = qn & 1u, sph = (qn >> 1) & 1u;
-      int32_t* sel = sel2 + slot * kMaxTopk;
+      int32_t* sel = sel2 + (slot % C::SEL_BUFS) * kMaxTopk;
       int32_t total = 0;
       if (group_a) {
         if (!gate(info_empty(slot), sph ^ 1u, 10)) break;
+        // with one index list, the previous query's list must be fully read: its last reader,
+        // the output-ring group, arrives on that query's info_empty after its gathers
+        if (C::SEL_BUFS == 1 && qn >= 1 && !gate(info_empty((qn - 1) & 1u), ((qn - 1) >> 1) & 1u, 15)) break;
         // ---- compact the valid entries of the index row, preserving their order
         const int32_t* row = p.idx + static_cast<size_t>(qi) * p.topk;
         const int32_t j0 = min(static_cast<int32_t>(gtid) * per, p.topk), j1 = min(j0 + per, p.topk);
