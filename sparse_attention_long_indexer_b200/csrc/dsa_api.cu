@@ -63,6 +63,7 @@ namespace {
 
 constexpr uint64_t kWaitBudgetNs = 2000000000ull;   // 2 s per bounded wait
 constexpr size_t kAlign = 256;
+constexpr int kPrefillNQ = 4;                       // queries per prefill indexer work item
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -148,8 +149,8 @@ DeviceInfo device_info() {
     cache[dev].sms = sms;
     cache[dev].sm100 = (major == 10 && minor == 0);
     // per-device kernel attributes (dynamic shared memory above 48 KB)
-    cudaFuncSetAttribute(indexer_topk_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         IdxCfg<4>::SMEM_BYTES);
+    cudaFuncSetAttribute(indexer_topk_kernel<kPrefillNQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         IdxCfg<kPrefillNQ>::SMEM_BYTES);
     cudaFuncSetAttribute(indexer_topk_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          IdxCfg<1>::SMEM_BYTES);
     cudaFuncSetAttribute(sparse_mla_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -264,12 +265,13 @@ dsa_status run_indexer(const dsa_dims& d, const uint8_t* q_idx, const __nv_bfloa
     return from_cuda(cudaGetLastError());
   }
   p.n_chunks = 0;
-  p.n_items = d.batch * ((d.n_q + 3) / 4);
+  p.n_items = d.batch * ((d.n_q + kPrefillNQ - 1) / kPrefillNQ);
   if (!encode_rows_u8(&map_q, q_idx, static_cast<uint64_t>(d.n_q) * kIdxHeads, static_cast<uint64_t>(d.batch),
-                      4 * kIdxHeads))
+                      kPrefillNQ * kIdxHeads))
     return DSA_ERR_CUDA;
   const int grid = std::min(p.n_items, dev.sms);
-  indexer_topk_kernel<4><<<grid, IdxCfg<4>::THREADS, IdxCfg<4>::SMEM_BYTES, st>>>(map_q, map_k, p);
+  indexer_topk_kernel<kPrefillNQ><<<grid, IdxCfg<kPrefillNQ>::THREADS, IdxCfg<kPrefillNQ>::SMEM_BYTES, st>>>(map_q,
+                                                                                                        map_k, p);
   return from_cuda(cudaGetLastError());
 }
 

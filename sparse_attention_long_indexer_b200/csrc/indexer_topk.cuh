@@ -35,14 +35,17 @@ namespace dsa {
 constexpr int kIdxHeads = 64;     // H_I (padded)
 constexpr int kIdxDim = 128;      // d_I (padded), one 128-byte row per head / key
 constexpr int kKeyTile = 128;     // keys per MMA tile (M)
-constexpr int kCand = 3584;       // candidate capacity per query
 constexpr int kDecodeChunk = 8192;  // keys per decode work item
 constexpr int kSyncTiles = 2;       // key tiles between two capacity checks of a candidate buffer
 
 template <int NQ>
 struct IdxCfg {
   static constexpr int N = NQ * kIdxHeads;                 // accumulator columns per tile
+  static constexpr int NBUF = (NQ == 2) ? 4 : 2;           // TMEM accumulators (NBUF * N <= 512)
   static constexpr int HALVES = (NQ == 4) ? 2 : 1;         // MMAs per tile (query pairs)
+  // few warps: registers for the head weights and all 64 head columns at once
+  static constexpr bool WIDE = NQ <= 2;
+  static constexpr int CAND = (NQ == 2) ? 6144 : 3584;     // candidate capacity per query
   static constexpr int NH = N / HALVES;                    // MMA N
   static constexpr int EPI_WARPS = 4 * NQ;                 // a query per group of 4 lane-quarter warps
   static constexpr int EPI_THREADS = EPI_WARPS * 32;
@@ -50,25 +53,26 @@ struct IdxCfg {
   static constexpr int PRODUCER_WARP = EPI_WARPS;
   static constexpr int MMA_WARP = EPI_WARPS + 1;
   static constexpr int THREADS = (EPI_WARPS + 2) * 32;
-  static constexpr int STAGES = (NQ == 4) ? 4 : 8;
+  static constexpr int STAGES = (NQ == 4) ? 4 : (NQ == 2) ? 6 : 8;
   static constexpr int Q_BYTES = NQ * kIdxHeads * kIdxDim;
   static constexpr int K_BYTES = kKeyTile * kIdxDim;       // 16 KB
-  static constexpr int TMEM_COLS = 2 * N;                  // two accumulators
-  static constexpr int MAXPER = kCand / GROUP_THREADS;
+  static constexpr int TMEM_COLS = NBUF * N;
+  static constexpr int MAXPER = CAND / GROUP_THREADS;
   // shared-memory layout (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_KEYS = OFF_K + STAGES * K_BYTES;
-  static constexpr int OFF_POS = OFF_KEYS + NQ * kCand * 4;
-  static constexpr int OFF_W = OFF_POS + NQ * kCand * 4;
+  static constexpr int OFF_POS = OFF_KEYS + NQ * CAND * 4;
+  static constexpr int OFF_W = OFF_POS + NQ * CAND * 4;
   static constexpr int OFF_SEL = OFF_W + NQ * kIdxHeads * 4;
   static constexpr int OFF_QST = OFF_SEL + NQ * static_cast<int>(sizeof(SelectScratch));
   static constexpr int OFF_BAR = (OFF_QST + 5 * 4 * NQ + 16 + 7) & ~7;
   static constexpr int NUM_BARS = 2 * STAGES + 2 + 8 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
-  static_assert(kCand % GROUP_THREADS == 0, "candidate buffer must split evenly");
-  static_assert(kCand - kSyncTiles * kKeyTile >= 2048, "a checked buffer must hold the largest k");
+  static_assert(CAND % GROUP_THREADS == 0 && MAXPER <= 64, "candidate buffer must split evenly");
+  static_assert(CAND - kSyncTiles * kKeyTile >= 2048, "a checked buffer must hold the largest k");
+  static_assert(NBUF * HALVES <= 4 && TMEM_COLS <= 512, "accumulators");
   static_assert(THREADS <= 1024 && NQ <= 4, "block shape");
   static_assert(Q_BYTES % 1024 == 0 && K_BYTES % 1024 == 0, "swizzle atoms");
 };
@@ -160,8 +164,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
   const uint32_t q_full = bar0 + 8u * (2 * C::STAGES);
   const uint32_t q_empty = q_full + 8;
   // accumulator buffer b, half h (queries 2h, 2h+1 of a 4-query block)
-  auto acc_full = [&](uint32_t b, uint32_t h) { return q_full + 16 + 8u * (2 * b + h); };
-  auto acc_empty = [&](uint32_t b, uint32_t h) { return q_full + 48 + 8u * (2 * b + h); };
+  auto acc_full = [&](uint32_t b, uint32_t h) { return q_full + 16 + 8u * (b * C::HALVES + h); };
+  auto acc_empty = [&](uint32_t b, uint32_t h) { return q_full + 48 + 8u * (b * C::HALVES + h); };
   const uint32_t mma_done = q_full + 80;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
@@ -174,7 +178,7 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (uint32_t b = 0; b < 2; ++b)
+    for (uint32_t b = 0; b < static_cast<uint32_t>(C::NBUF); ++b)
       for (uint32_t h = 0; h < static_cast<uint32_t>(C::HALVES); ++h) {
         mbar_init(acc_full(b, h), 1);
         mbar_init(acc_empty(b, h), C::EPI_WARPS / C::HALVES);
@@ -244,7 +248,7 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         qph ^= 1u;
         bool ok = true;
         for (int32_t t = 0; t < it.ntiles; ++t, ++g) {
-          const uint32_t buf = g & 1u, acc_ph = (g >> 1) & 1u;
+          const uint32_t buf = g % C::NBUF, acc_ph = (g / C::NBUF) & 1u;
           if (!wt.wait(k_full(stage), phase, 5)) { ok = false; break; }
           const uint32_t a_base = sbase + C::OFF_K + stage * C::K_BYTES;
           // one MMA group per query pair, each announced on its own, so the two epilogue
@@ -289,8 +293,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     const uint32_t lane_base = (quarter * 32u) << 16;
     SelectScratch* gsel = sel + q;
     volatile uint32_t* snap = q_strict + NQ + 2 * q;     // two parity slots per group
-    uint32_t* cq_keys = cand_keys + q * kCand;
-    int32_t* cq_pos = cand_pos + q * kCand;
+    uint32_t* cq_keys = cand_keys + q * C::CAND;
+    int32_t* cq_pos = cand_pos + q * C::CAND;
     uint32_t g = 0, nsync = 0;
     // One barrier per step: thread 0 of the group publishes the abort flag as it sees it into
     // a parity slot before the barrier and the group reads that slot after it. A slot is
@@ -324,6 +328,12 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       named_barrier(bar_id, C::GROUP_THREADS);
       const int32_t qpos = q_valid ? it.len - p.n_q + i : -1;
       const float4* w4 = reinterpret_cast<const float4*>(wq + q * kIdxHeads);
+      // with few epilogue warps the query's head weights stay in registers for the whole item
+      float2 wr[C::WIDE ? kIdxHeads / 2 : 1];
+      if constexpr (C::WIDE) {
+#pragma unroll
+        for (int h = 0; h < kIdxHeads / 2; ++h) wr[h] = reinterpret_cast<const float2*>(wq + q * kIdxHeads)[h];
+      }
       const float* ks_row = p.k_scale + static_cast<size_t>(it.b) * p.max_len;
       const int32_t s_lane = it.s_begin + static_cast<int32_t>(quarter * 32 + lane);
       // the key scale of the next tile is loaded one tile ahead (clamped address; the value
@@ -333,7 +343,7 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       };
       float ks_next = key_scale(0);
       for (int32_t t = 0; t < it.ntiles; ++t, ++g) {
-        const uint32_t buf = g & 1u, acc_ph = (g >> 1) & 1u;
+        const uint32_t buf = g % C::NBUF, acc_ph = (g / C::NBUF) & 1u;
         const int32_t s = s_lane + t * kKeyTile;
         const bool in_range = s < it.s_end;
         const float ks = ks_next;
@@ -341,14 +351,33 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         // every lane waits (no divergent branch); the warp then runs the collective TMEM loads
         const bool ok = __all_sync(0xffffffffu, wt.wait(acc_full(buf, half), acc_ph, 8)) != 0;
         if (ok) {
-          uint32_t x[32];
           tc_fence_after();
           const uint32_t col = buf * C::N + q * kIdxHeads;
-          // sum_j w'_j * ReLU(x_j): packed fp32x2 FMAs over 4 independent accumulator pairs; the
-          // 64 head columns come in two loads of 32 (fewer live registers), and the accumulator
-          // is released after the second
+          // sum_j w'_j * ReLU(x_j): packed fp32x2 FMAs over 4 independent accumulator pairs (head
+          // h goes to pair 2*((h/4)&1) + ((h/2)&1), the same in both forms below)
           float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                            make_float2(0.f, 0.f)};
+          if constexpr (C::WIDE) {
+            // all 64 head columns in one go, weights from registers
+            uint32_t x[64];
+            tmem_ld32(tmem + lane_base + col, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+            tmem_ld32(tmem + lane_base + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty(buf, half));
+#pragma unroll
+            for (int h = 0; h < kIdxHeads; h += 4) {
+              const float2 r01 = make_float2(fmaxf(__uint_as_float(x[h + 0]), 0.f), fmaxf(__uint_as_float(x[h + 1]), 0.f));
+              const float2 r23 = make_float2(fmaxf(__uint_as_float(x[h + 2]), 0.f), fmaxf(__uint_as_float(x[h + 3]), 0.f));
+              const int c = (h / 4) & 1;
+              acc[2 * c] = __ffma2_rn(wr[h / 2], r01, acc[2 * c]);
+              acc[2 * c + 1] = __ffma2_rn(wr[h / 2 + 1], r23, acc[2 * c + 1]);
+            }
+          } else {
+          // the 64 head columns come in two loads of 32 (fewer live registers), and the
+          // accumulator is released after the second
+          uint32_t x[32];
 #pragma unroll
           for (int part = 0; part < 2; ++part) {
             tmem_ld32(tmem + lane_base + col + 32 * part, x);
@@ -367,6 +396,7 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
               acc[2 * c] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc[2 * c]);
               acc[2 * c + 1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc[2 * c + 1]);
             }
+          }
           }
           const float score =
               (((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y))) * ks;
@@ -387,17 +417,17 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
           }
         }
         // capacity check every kSyncTiles tiles: between two checks at most kSyncTiles * 128
-        // candidates arrive, and a check leaves at most kCand - kSyncTiles * 128
+        // candidates arrive, and a check leaves at most CAND - kSyncTiles * 128
         if (t % kSyncTiles != kSyncTiles - 1 && t + 1 != it.ntiles) continue;
         if (uniform_stop()) { stop = true; break; }
         const uint32_t n = q_count[q];
-        if (n > static_cast<uint32_t>(kCand - kSyncTiles * kKeyTile)) {
+        if (n > static_cast<uint32_t>(C::CAND - kSyncTiles * kKeyTile)) {
           // cheap range-histogram shrink; the exact select only if it frees too little
           uint32_t thr = 0;
           const uint32_t m = shrink_candidates<C::GROUP_THREADS, C::MAXPER>(
               cq_keys, cq_pos, n, static_cast<uint32_t>(p.topk), gsel, gtid, bar_id, &thr);
           // the exact select when the shrink freed less than half of the usable space
-          if (m > static_cast<uint32_t>(kCand - kSyncTiles * kKeyTile + p.topk) / 2) {
+          if (m > static_cast<uint32_t>(C::CAND - kSyncTiles * kKeyTile + p.topk) / 2) {
             const uint32_t vk = select_exact<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, m,
                                                                           static_cast<uint32_t>(p.topk), gsel, gtid,
                                                                           bar_id);

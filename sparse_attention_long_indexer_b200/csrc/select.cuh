@@ -182,13 +182,14 @@ template <int T, int MAXPER, typename Keep>
 __device__ __forceinline__ void compact_candidates(uint32_t* keys, int32_t* pos, const uint32_t (&rk)[MAXPER],
                                                    const int32_t (&rp)[MAXPER], Keep keep, SelectScratch* sc,
                                                    uint32_t bar_id) {
-  static_assert(MAXPER <= 32, "keep mask");
+  static_assert(MAXPER <= 64, "keep mask");
   const uint32_t lane = threadIdx.x & 31;
-  uint32_t mask = 0, c = 0;
+  uint64_t mask = 0;
+  uint32_t c = 0;
 #pragma unroll
   for (int j = 0; j < MAXPER; ++j)
     if (rp[j] >= 0 && keep(rk[j], rp[j])) {
-      mask |= 1u << j;
+      mask |= 1ull << j;
       ++c;
     }
   uint32_t incl = c;
@@ -203,7 +204,7 @@ __device__ __forceinline__ void compact_candidates(uint32_t* keys, int32_t* pos,
   uint32_t at = base + incl - c;
 #pragma unroll
   for (int j = 0; j < MAXPER; ++j)
-    if (mask & (1u << j)) {
+    if (mask & (1ull << j)) {
       keys[at] = rk[j];
       pos[at] = rp[j];
       ++at;
