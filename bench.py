@@ -269,8 +269,8 @@ def run_ours(args, cfg, rank, world, local_rank):
 
 
 
-def run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
-    """Same step, inputs copied from pinned host memory and results read back every step."""
+def run_e2e_whole(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
+    """Same step, inputs copied from pinned host memory and results read back every step, as one call."""
     names = ["q_idx", "w", "k_idx", "q", "kv", "lengths"]
     try:
         host = {k: torch.empty(g[k].shape, dtype=g[k].dtype, pin_memory=True) for k in names}
@@ -320,6 +320,122 @@ def run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
             "pinned": pinned}
 
 
+def run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
+    """The step end to end through the public API: inputs from pinned host memory, results read back.
+
+    A prefill sequence (B = 1) runs as query chunks so that transfers overlap compute: the key-side
+    inputs (k_idx, latent_kv, key scales) go up first, then each chunk's query-side inputs go up on a
+    copy stream, its dsa_forward runs on the compute stream and its out, lse and idx come back on a
+    second copy stream, through a ring of device buffers. A chunk of queries [i0, i1) is the call with
+    n_q = i1 - i0 and lengths = i1, the query positions the header defines; it computes exactly what
+    the whole call computes for those queries.
+    """
+    if cfg.batch != 1 or args.e2e_chunk <= 0:
+        return run_e2e_whole(args, cfg, dsa, dims, g, scales, ws, dev, stream, world)
+    L, H, dv, k = cfg.max_len, cfg.n_heads, cfg.d_v, cfg.topk
+    C = min(args.e2e_chunk, cfg.n_q)
+    starts = list(range(0, cfg.n_q, C))
+    NS = 3                                               # device buffer slots
+    q_side = ["q_idx", "w", "q"]
+    try:
+        host = {n: torch.empty(g[n].shape, dtype=g[n].dtype, pin_memory=True) for n in q_side + ["k_idx", "kv"]}
+        host_scales = torch.empty(scales.shape, dtype=scales.dtype, pin_memory=True)
+        host_out = torch.empty((1, cfg.n_q, H, dv), dtype=torch.bfloat16, pin_memory=True)
+        host_lse = torch.empty((1, cfg.n_q, H), dtype=torch.float32, pin_memory=True)
+        host_idx = torch.empty((1, cfg.n_q, k), dtype=torch.int32, pin_memory=True)
+    except RuntimeError:
+        return {"value": None, "unit": UNIT, "note": "pinned host allocation failed"}
+    for n in host:
+        host[n].copy_(g[n])
+    host_scales.copy_(scales)
+    nq = cfg.n_q
+    # device: key side once, query side and outputs per slot
+    d_kidx, d_kv = torch.empty_like(g["k_idx"]), torch.empty_like(g["kv"])
+    d_kscale = torch.empty(L, dtype=torch.float32, device=dev)
+    # query-side tensors as [n_q, row] (B = 1): a chunk is a row range
+    hrow = {n: host[n].view(nq, -1) for n in q_side}
+    slot = [dict({n: torch.empty((C, hrow[n].shape[1]), dtype=hrow[n].dtype, device=dev) for n in q_side},
+                 scales=torch.empty(C + L, dtype=torch.float32, device=dev),
+                 out=torch.empty((C, H * dv), dtype=torch.bfloat16, device=dev),
+                 lse=torch.empty((C, H), dtype=torch.float32, device=dev),
+                 idx=torch.empty((C, k), dtype=torch.int32, device=dev)) for _ in range(NS)]
+    hout, hlse, hidx = host_out.view(nq, -1), host_lse.view(nq, -1), host_idx.view(nq, -1)
+    ends = torch.tensor([min(i0 + C, nq) + (L - nq) for i0 in starts], dtype=torch.int32, device=dev)
+    chunk_dims = {}
+    for i0 in starts:
+        c = min(C, nq - i0)
+        if c not in chunk_dims:
+            chunk_dims[c] = dsa.make_dims(1, c, L, cfg.n_idx_heads, cfg.idx_dim, H, cfg.d_latent, cfg.d_rope,
+                                          cfg.softmax_scale)
+    ws_c = dsa.Workspace.create(chunk_dims[C], k, device=dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    h2d = (sum(host[n].numel() * host[n].element_size() for n in host) + host_scales.numel() * 4)
+    d2h = host_out.numel() * 2 + host_lse.numel() * 4 + host_idx.numel() * 4
+
+    def ev():
+        return torch.cuda.Event()
+
+    prev = {"keys_free": None, "comp": [None] * NS, "d2h": [None] * NS}
+
+    def step():
+        with torch.cuda.stream(s_in):
+            if prev["keys_free"] is not None:
+                s_in.wait_event(prev["keys_free"])
+            d_kidx.copy_(host["k_idx"], non_blocking=True)
+            d_kv.copy_(host["kv"], non_blocking=True)
+            d_kscale.copy_(host_scales[nq:], non_blocking=True)
+        last = None
+        for ci, i0 in enumerate(starts):
+            c, sl = min(C, nq - i0), ci % NS
+            bufs = slot[sl]
+            with torch.cuda.stream(s_in):
+                if prev["comp"][sl] is not None:
+                    s_in.wait_event(prev["comp"][sl])      # the slot's inputs are no longer read
+                for n in q_side:
+                    bufs[n][:c].copy_(hrow[n][i0:i0 + c], non_blocking=True)
+                bufs["scales"][:c].copy_(host_scales[i0:i0 + c], non_blocking=True)
+                bufs["scales"][c:c + L].copy_(d_kscale, non_blocking=True)
+                ready = ev()
+                ready.record(s_in)
+            stream.wait_event(ready)
+            if prev["d2h"][sl] is not None:
+                stream.wait_event(prev["d2h"][sl])         # the slot's outputs have been read back
+            dsa.dsa_forward(chunk_dims[c], bufs["q_idx"][:c], bufs["w"][:c], d_kidx, bufs["scales"][:c + L],
+                            ends[ci:ci + 1], k, bufs["q"][:c], d_kv, bufs["idx"][:c], bufs["out"][:c],
+                            bufs["lse"][:c], ws_c.buf, stream)
+            done = ev()
+            done.record(stream)
+            prev["comp"][sl] = done
+            last = done
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done)
+                hout[i0:i0 + c].copy_(bufs["out"][:c], non_blocking=True)
+                hlse[i0:i0 + c].copy_(bufs["lse"][:c], non_blocking=True)
+                hidx[i0:i0 + c].copy_(bufs["idx"][:c], non_blocking=True)
+                back = ev()
+                back.record(s_out)
+                prev["d2h"][sl] = back
+        prev["keys_free"] = last
+
+    steps = max(1, min(args.steps, args.e2e_steps))
+    step()
+    torch.cuda.synchronize(dev)
+    ws_c.check()
+    if world > 1:
+        torch.distributed.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s_in)
+    for _ in range(steps):
+        step()
+    b.record(s_out)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(a.elapsed_time(b), dev)
+    ws_c.check()
+    return {"value": aggregate_value(cfg.batch * cfg.n_q, steps, world, ms), "unit": UNIT, "steps": steps,
+            "ms_per_step": ms / steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "pinned": True,
+            "chunk_queries": C, "streams": "h2d / compute / d2h overlapped"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -329,6 +445,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-chunk", type=int, default=8192,
+                    help="queries per dsa_forward call in the e2e measurement (0 = one call per step)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)

@@ -201,3 +201,38 @@ def test_empty_problem_is_a_no_op():
     e = torch.empty(0, device="cuda")
     dsa.dsa_forward(dims, e, e, e, e, e, cfg.topk, e, e, None, e, e, ws.buf)
     ws.check()
+
+
+# ----------------------------------------------------------------------------- query chunks
+def test_query_chunks_match_one_call():
+    """A prefill sequence run as query chunks [i0, i1) (n_q = i1 - i0, lengths = i1) gives what one
+    call over all queries gives, query by query (the e2e measurement runs the step this way)."""
+    cfg = synthetic.config("prefill_4k")
+    g = _inputs(cfg, 5)
+    idx, out, lse = _run_forward(cfg, g)
+    L, C = cfg.max_len, 1024
+    c_idx, c_out, c_lse = torch.empty_like(idx), torch.empty_like(out), torch.empty_like(lse)
+    dims_c = dsa.make_dims(1, C, L, cfg.n_idx_heads, cfg.idx_dim, cfg.n_heads, cfg.d_latent, cfg.d_rope,
+                           cfg.softmax_scale)
+    ws = dsa.Workspace.create(dims_c, cfg.topk)
+    q_scale = g["q_scale"].reshape(-1)
+    k_scale = g["k_scale"].reshape(-1).float()
+    for i0 in range(0, cfg.n_q, C):
+        scales = torch.cat([q_scale[i0:i0 + C].float(), k_scale]).contiguous()
+        lengths = torch.tensor([i0 + C], dtype=torch.int32, device="cuda")
+        o_i, o_o, o_l = (torch.empty((1, C, cfg.topk), dtype=torch.int32, device="cuda"),
+                         torch.empty((1, C, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device="cuda"),
+                         torch.empty((1, C, cfg.n_heads), dtype=torch.float32, device="cuda"))
+        dsa.dsa_forward(dims_c, g["q_idx"][:, i0:i0 + C].contiguous(), g["w"][:, i0:i0 + C].contiguous(), g["k_idx"],
+                        scales, lengths, cfg.topk, g["q"][:, i0:i0 + C].contiguous(), g["kv"], o_i, o_o, o_l, ws.buf)
+        c_idx[:, i0:i0 + C], c_out[:, i0:i0 + C], c_lse[:, i0:i0 + C] = o_i, o_o, o_l
+    torch.cuda.synchronize()
+    ws.check()
+    # the same index sets; their order within a row is unspecified (candidate appends from four warps
+    # interleave), and it sets the summation order and where the softmax rescales, so out may differ
+    # by the rounding of P and of the sums: within the parity tolerances of the attention
+    assert torch.equal(torch.sort(idx, dim=-1).values, torch.sort(c_idx, dim=-1).values)
+    a, b = out.float(), c_out.float()
+    assert (a - b).abs().max().item() <= 1e-2
+    assert ((a - b).norm() / a.norm()).item() <= 5e-3
+    assert (lse - c_lse).abs().max().item() <= 2e-3
