@@ -445,7 +445,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=2)
-    ap.add_argument("--e2e-chunk", type=int, default=8192,
+    ap.add_argument("--e2e-chunk", type=int, default=4096,
                     help="queries per dsa_forward call in the e2e measurement (0 = one call per step)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
