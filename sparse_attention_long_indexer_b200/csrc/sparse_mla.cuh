@@ -57,12 +57,12 @@ struct AttnCfg {
   static constexpr int SB_BYTES = 9 * SB_ATOM;           // own 32 rows x 576 dims
   static constexpr int VR_ATOM = kBlk * 128;             // 64 rows x 128 B
   static constexpr int VR_BYTES = 4 * VR_ATOM;           // 64 rows x this CTA's 256 output dims
-  static constexpr int Q_TMEM_DIMS = 384;                // dims 0..383 of q in TMEM, the rest in smem
+  static constexpr int Q_TMEM_DIMS = 320;                // dims 0..319 of q in TMEM, the rest in smem
   static constexpr int QS_ATOMS = (kDqk - Q_TMEM_DIMS) / 64;
   static constexpr int QS_BYTES = QS_ATOMS * 64 * 128;   // 64 heads x dims 384..575
   static constexpr int P_BYTES = 64 * 128;               // 64 heads x 64 rows bf16
-  static constexpr int P_BUFS = 1;                       // P of consecutive blocks (1 or 2)
-  static constexpr int S_BUFS = 2;                       // TMEM logits buffers
+  static constexpr int P_BUFS = 2;                       // P of consecutive blocks (1 or 2)
+  static constexpr int S_BUFS = 3;                       // TMEM logits buffers
   static constexpr int SOFTMAX_WARPS = 4;
   static constexpr int PRODUCER_WARPS = 8;               // 4 gather the logits ring, 4 the output ring
   static constexpr int GROUP_WARPS = PRODUCER_WARPS / 2;
@@ -77,9 +77,7 @@ struct AttnCfg {
   static constexpr int OFF_VR = OFF_SB + SB_STAGES * SB_BYTES;
   static constexpr int OFF_QS = OFF_VR + VR_STAGES * VR_BYTES;
   static constexpr int OFF_P = OFF_QS + QS_BYTES;
-  static constexpr int SEL_BUFS = 2;                     // compacted index lists (1 or 2)
-  static constexpr int OFF_SEL = OFF_P + P_BUFS * P_BYTES;         // SEL_BUFS x kMaxTopk indices
-  static constexpr int OFF_XMAX = OFF_SEL + SEL_BUFS * kMaxTopk * 4;  // 2 x 128 floats
+  static constexpr int OFF_XMAX = OFF_P + P_BUFS * P_BYTES;        // 2 x 128 floats
   static constexpr int OFF_SCAN = OFF_XMAX + 2 * 128 * 4;
   static constexpr int OFF_INFO = OFF_SCAN + 64;
   static constexpr int OFF_BAR = OFF_INFO + 16;
@@ -140,7 +138,6 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  int32_t* sel2 = reinterpret_cast<int32_t*>(smem + C::OFF_SEL);
   float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
   int32_t* scan = reinterpret_cast<int32_t*>(smem + C::OFF_SCAN);
   int32_t* info = reinterpret_cast<int32_t*>(smem + C::OFF_INFO);
@@ -244,7 +241,6 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     const uint32_t gw = pw % C::GROUP_WARPS;           // warp in group = TMEM lane quarter (group A)
     const uint32_t gtid = ptid % C::GROUP_THREADS;
     volatile int32_t* go = scan + 8;
-    const int32_t per = (p.topk + C::GROUP_THREADS - 1) / C::GROUP_THREADS;
     uint32_t qn = 0, nsync = 0, qq = 0;
     uint32_t st = 0, ph = 0;                            // ring position (this group's ring)
     const uint32_t n_stages = group_a ? C::SB_STAGES : C::VR_STAGES;
@@ -261,42 +257,26 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     };
     for (int32_t qi = cid; qi < p.n_queries; qi += ncl, ++qn) {
       const uint32_t slot = qn & 1u, sph = (qn >> 1) & 1u;
-      int32_t* sel = sel2 + (slot % C::SEL_BUFS) * kMaxTopk;
-      int32_t total = 0;
+      const int32_t* idx_row = p.idx + static_cast<size_t>(qi) * p.topk;
+      int32_t total = 0;                                 // extent of the index row (see below)
       if (group_a) {
         if (!gate(info_empty(slot), sph ^ 1u, 10)) break;
-        // with one index list, the previous query's list must be fully read: its last reader,
-        // the output-ring group, arrives on that query's info_empty after its gathers
-        if (C::SEL_BUFS == 1 && qn >= 1 && !gate(info_empty((qn - 1) & 1u), ((qn - 1) >> 1) & 1u, 15)) break;
-        // ---- compact the valid entries of the index row, preserving their order
-        const int32_t* row = p.idx + static_cast<size_t>(qi) * p.topk;
-        const int32_t j0 = min(static_cast<int32_t>(gtid) * per, p.topk), j1 = min(j0 + per, p.topk);
-        int32_t cnt = 0;
-        for (int32_t j = j0; j < j1; ++j) {
-          const int32_t v = __ldg(row + j);
+        // ---- the extent of the index row: one past its last valid entry. Entries < 0 (padding)
+        // and >= max_len (reported) are masked wherever they appear: their rows are gathered as
+        // zeros and their logits set to -inf, so blocks are read straight from the index row.
+        int32_t last = -1;
+        for (int32_t j = static_cast<int32_t>(gtid); j < p.topk; j += C::GROUP_THREADS) {
+          const int32_t v = __ldg(idx_row + j);
           if (v >= p.max_len) record_error(p.status, DSA_ERR_INDEX_RANGE, static_cast<uint32_t>(qi));
-          cnt += (v >= 0 && v < p.max_len) ? 1 : 0;
+          if (v >= 0 && v < p.max_len) last = j;
         }
-        int32_t incl = cnt;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (static_cast<int32_t>(lane) >= o) incl += v;
-        }
-        if (lane == 31) scan[gw] = incl;
+        for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+        if (lane == 0) scan[gw] = last;
         named_barrier(2, C::GROUP_THREADS);
-        int32_t base = incl - cnt;
         total = 0;
 #pragma unroll
-        for (int w = 0; w < C::GROUP_WARPS; ++w) {
-          base += (w < static_cast<int>(gw)) ? scan[w] : 0;
-          total += scan[w];
-        }
-        for (int32_t j = j0; j < j1; ++j) {
-          const int32_t v = __ldg(row + j);
-          if (v >= 0 && v < p.max_len) sel[base++] = v;
-        }
-        named_barrier(2, C::GROUP_THREADS);
+        for (int w = 0; w < C::GROUP_WARPS; ++w) total = max(total, scan[w] + 1);
         if (gtid == 0) {
           info[slot] = total;
           mbar_arrive(info_full(slot));
@@ -348,6 +328,26 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         const uint32_t cc = gtid & 7u, r0 = gtid >> 3;
         const int32_t own0 = 32 * static_cast<int32_t>(rank);
         const uint32_t seg0 = 128u * rank;               // group B: segments 2r, 2r+1, 4+2r, 5+2r
+        // block row r of block b: its row of the latent cache, or -1 when masked (padding, past the
+        // extent, or out of range); read from the index row one block ahead of its gathers
+        constexpr int RS = C::GROUP_THREADS / 8;       // rows per pass
+        constexpr int NRA = 32 / RS, NRB = kBlk / RS;  // rows per thread: logits ring, output ring
+        auto row_of = [&](int32_t b, int32_t r) -> int32_t {
+          const int32_t j = b * kBlk + r;
+          const int32_t v = j < total ? __ldg(idx_row + j) : -1;
+          return (v >= 0 && v < p.max_len) ? v : -1;
+        };
+        int32_t rows_a[NRA], rows_b[NRB];
+        auto load_rows = [&](int32_t b) {
+          if (group_a) {
+#pragma unroll
+            for (int q = 0; q < NRA; ++q) rows_a[q] = row_of(b, own0 + static_cast<int32_t>(r0) + RS * q);
+          } else {
+#pragma unroll
+            for (int q = 0; q < NRB; ++q) rows_b[q] = row_of(b, static_cast<int32_t>(r0) + RS * q);
+          }
+        };
+        load_rows(0);
         int32_t pending = -1;
         auto announce = [&](int32_t stage) {
           fence_proxy_async_smem();
@@ -368,34 +368,20 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
           if (!warp_wait(empty_bar, ph ^ 1u, 11)) { ok = false; break; }
           if (group_a) {
             const uint32_t dst0 = sbase + C::OFF_SB + st * C::SB_BYTES + sw128_offset(r0, cc);
-            constexpr int RS = C::GROUP_THREADS / 8;       // rows per pass
-            int32_t rows[32 / RS];
 #pragma unroll
-            for (int q = 0; q < 32 / RS; ++q) {
-              const int32_t j = b * kBlk + own0 + static_cast<int32_t>(r0) + RS * q;
-              rows[q] = j < total ? sel[j] : -1;
-            }
-#pragma unroll
-            for (int q = 0; q < 32 / RS; ++q) {
-              const bool v = rows[q] >= 0;
-              const __nv_bfloat16* src = (v ? kv_seq + static_cast<size_t>(rows[q]) * kDqk : p.kv) + cc * 8;
+            for (int q = 0; q < NRA; ++q) {
+              const bool v = rows_a[q] >= 0;
+              const __nv_bfloat16* src = (v ? kv_seq + static_cast<size_t>(rows_a[q]) * kDqk : p.kv) + cc * 8;
               const uint32_t n = v ? 16u : 0u;
 #pragma unroll
               for (int a = 0; a < 9; ++a) cp_async_16(dst0 + q * RS * 128 + a * C::SB_ATOM, src + a * 64, n);
             }
           } else {
             const uint32_t dst0 = sbase + C::OFF_VR + st * C::VR_BYTES + sw128_offset(r0, cc);
-            constexpr int RS = C::GROUP_THREADS / 8;       // rows per pass
-            int32_t rows[kBlk / RS];
 #pragma unroll
-            for (int q = 0; q < kBlk / RS; ++q) {
-              const int32_t j = b * kBlk + static_cast<int32_t>(r0) + RS * q;
-              rows[q] = j < total ? sel[j] : -1;
-            }
-#pragma unroll
-            for (int q = 0; q < kBlk / RS; ++q) {
-              const bool v = rows[q] >= 0;
-              const __nv_bfloat16* src = (v ? kv_seq + static_cast<size_t>(rows[q]) * kDqk : p.kv) + seg0 + cc * 8;
+            for (int q = 0; q < NRB; ++q) {
+              const bool v = rows_b[q] >= 0;
+              const __nv_bfloat16* src = (v ? kv_seq + static_cast<size_t>(rows_b[q]) * kDqk : p.kv) + seg0 + cc * 8;
               const uint32_t n = v ? 16u : 0u;
               const uint32_t d = dst0 + q * RS * 128;
               cp_async_16(d + 0 * C::VR_ATOM, src + 0, n);
@@ -405,6 +391,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
             }
           }
           cp_async_commit();
+          if (b + 1 < n_blocks) load_rows(b + 1);
           if (pending >= 0) {
             cp_async_wait<1>();
             announce(pending);
@@ -415,7 +402,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         cp_async_wait<0>();
         if (pending >= 0) announce(pending);
       }
-      if (!group_a) {                                  // sel[slot] no longer read by this warp
+      if (!group_a) {                                  // info[slot] no longer read by this warp
         __syncwarp();
         if (lane == 0) mbar_arrive(info_empty(slot));
       }
@@ -569,7 +556,17 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         continue;
       }
       float m2 = -INFINITY, l = 0.f;
+      // validity of this half's 32 rows of a block: lane j reads entry 32*half + j of the block from
+      // the index row, one block ahead, and a ballot gives the mask (bit j: row j is attended)
+      const int32_t* idx_row = p.idx + static_cast<size_t>(qi) * p.topk;
+      auto entry = [&](int32_t b) -> int32_t {
+        const int32_t j = b * kBlk + 32 * static_cast<int32_t>(half) + static_cast<int32_t>(lane);
+        return j < total ? __ldg(idx_row + j) : -1;
+      };
+      int32_t e_next = entry(0);
       for (int32_t b = 0; b < n_blocks && ok; ++b) {
+        const uint32_t vmask = __ballot_sync(0xffffffffu, e_next >= 0 && e_next < p.max_len);
+        if (b + 1 < n_blocks) e_next = entry(b + 1);
         // ---- this lane's 32 logits
         if (lane == 0) got = wt.wait(s_full(s_i), s_u & 1u, 32) ? 1u : 0u;
         if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
@@ -580,12 +577,11 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         tc_fence_before();
         __syncwarp();
         if (++s_i == static_cast<uint32_t>(C::S_BUFS)) { s_i = 0; ++s_u; }
-        const int32_t nvalid = min(32, total - b * kBlk - 32 * static_cast<int32_t>(half));
         float z[32];
         float mb = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          z[j] = (j < nvalid) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
+          z[j] = ((vmask >> j) & 1u) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
           mb = fmaxf(mb, z[j]);
         }
         mb = fmaxf(mb, swap_partner(mb));
