@@ -577,13 +577,19 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         tc_fence_before();
         __syncwarp();
         if (++s_i == static_cast<uint32_t>(C::S_BUFS)) { s_i = 0; ++s_u; }
-        float z[32];
-        float mb = -INFINITY;
+        // masked logits become -inf (their P is then exactly 0); a block of all-valid rows, the
+        // usual case, skips the selects. The scale is positive, so the max of the raw logits
+        // times the scale is the max of the scaled ones.
+        const float sc = p.scale_log2;
+        if (vmask != 0xffffffffu) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          z[j] = ((vmask >> j) & 1u) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
-          mb = fmaxf(mb, z[j]);
+          for (int j = 0; j < 32; ++j)
+            if (!((vmask >> j) & 1u)) sr[j] = __float_as_uint(-INFINITY);
         }
+        float mraw = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) mraw = fmaxf(mraw, __uint_as_float(sr[j]));
+        float mb = mraw * sc;
         mb = fmaxf(mb, swap_partner(mb));
         if (!ok) break;
         const bool need = (mb > m2 + 8.0f);
@@ -593,16 +599,21 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
           m2 = mb;
           l *= alpha;
         }
+        // P = 2^(s*sc - m2) in bf16 for the output product; the row sum adds the same bf16 values,
+        // so the normalisation matches the weights the output product uses
         uint32_t pk[16];
-        float lsum = 0.f;
+        float2 lsum2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(ex2_approx(z[2 * j] - m2), ex2_approx(z[2 * j + 1] - m2));
+          const float e0 = ex2_approx(fmaf(__uint_as_float(sr[2 * j]), sc, -m2));
+          const float e1 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 1]), sc, -m2));
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
           const float2 back = __bfloat1622float2(pr);
-          lsum += back.x + back.y;
+          lsum2.x += back.x;
+          lsum2.y += back.y;
           pk[j] = *reinterpret_cast<const uint32_t*>(&pr);
         }
-        l += lsum;
+        l += lsum2.x + lsum2.y;
         // ---- the P buffer of block pb is free once the output MMA of block pb - P_BUFS has
         // finished; a rescale of O needs the one of block pb-1 finished (it implies the earlier ones)
         const bool rescale = __any_sync(0xffffffffu, need) && b > 0;
