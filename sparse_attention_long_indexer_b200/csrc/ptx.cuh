@@ -117,6 +117,30 @@ struct Waiter {
       }
     }
   }
+
+  // Wait until the 64-bit shared word at `addr` carries `tag` in its high half and return its
+  // low half. The writer stores tag and value in one aligned 64-bit store, so the pair is seen
+  // whole and needs no separate release/acquire.
+  __device__ __forceinline__ bool wait_tagged(uint32_t addr, uint32_t tag, uint32_t ptag, uint32_t& value) {
+    uint64_t w;
+    asm volatile("ld.volatile.shared.u64 %0, [%1];" : "=l"(w) : "r"(addr) : "memory");
+    if (static_cast<uint32_t>(w >> 32) == tag) { value = static_cast<uint32_t>(w); return true; }
+    const uint64_t t0 = global_timer_ns();
+    uint32_t spins = 0;
+    while (true) {
+      asm volatile("ld.volatile.shared.u64 %0, [%1];" : "=l"(w) : "r"(addr) : "memory");
+      if (static_cast<uint32_t>(w >> 32) == tag) { value = static_cast<uint32_t>(w); return true; }
+      if ((++spins & 63u) == 0) {
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > budget_ns) {
+          record_error(status, DSA_ERR_DEVICE_TIMEOUT, (where << 16) | ptag);
+          *abort = 1;
+          __threadfence_block();
+          return false;
+        }
+      }
+    }
+  }
 };
 
 // ------------------------------------------------------------------------- TMA (tiled, no swizzle choice here: the map carries it)

@@ -77,8 +77,8 @@ struct AttnCfg {
   static constexpr int OFF_VR = OFF_SB + SB_STAGES * SB_BYTES;
   static constexpr int OFF_QS = OFF_VR + VR_STAGES * VR_BYTES;
   static constexpr int OFF_P = OFF_QS + QS_BYTES;
-  static constexpr int OFF_XMAX = OFF_P + P_BUFS * P_BYTES;        // 2 x 128 floats
-  static constexpr int OFF_SCAN = OFF_XMAX + 2 * 128 * 4;
+  static constexpr int OFF_XMAX = OFF_P + P_BUFS * P_BYTES;        // 2 x 128 tagged words
+  static constexpr int OFF_SCAN = OFF_XMAX + 2 * 128 * 8;
   static constexpr int OFF_INFO = OFF_SCAN + 64;
   static constexpr int OFF_BAR = OFF_INFO + 16;
   static constexpr int NUM_BARS = 40;
@@ -138,7 +138,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
+  uint64_t* xmax = reinterpret_cast<uint64_t*>(smem + C::OFF_XMAX);
   int32_t* scan = reinterpret_cast<int32_t*>(smem + C::OFF_SCAN);
   int32_t* info = reinterpret_cast<int32_t*>(smem + C::OFF_INFO);
   const uint32_t bar0 = sbase + C::OFF_BAR;
@@ -153,7 +153,6 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
   auto s_full = [&](uint32_t i) { return B(31 + i); };   // commit: logits buffer i ready (3)
   auto p_empty = [&](uint32_t j) { return B(34 + j); };  // commit: output MMA that read P buffer j done (2)
   const uint32_t o_full = B(14);                         // commit: all output MMAs of a query done
-  auto pair_bar = [&](int w, int par) { return B(15 + 2 * w + par); };   // softmax warp pairs
   // barriers of the even CTA, arrived on by both CTAs
   auto sb_full2 = [&](int s) { return B(19 + s); };
   auto vr_full2 = [&](int s) { return B(22 + s); };
@@ -196,8 +195,6 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     }
     for (uint32_t j = 0; j < static_cast<uint32_t>(C::P_BUFS); ++j) mbar_init(p_empty(j), 1);
     mbar_init(o_full, 1);
-    for (int w = 0; w < 2; ++w)
-      for (int par = 0; par < 2; ++par) mbar_init(pair_bar(w, par), 2);
     mbar_init(q_full2, 2 * (1 + C::GROUP_WARPS));
     for (uint32_t j = 0; j < static_cast<uint32_t>(C::P_BUFS); ++j) {
       mbar_init(p_full2(j), C::SOFTMAX_WARPS + 1);
@@ -208,6 +205,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     *abort_flag = 0;
     fence_mbar_init();
   }
+  for (uint32_t i = threadIdx.x; i < 256u; i += blockDim.x) xmax[i] = 0;   // exchange numbers start at 1
   if (warp == C::MMA_WARP) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(C::TMEM_COLS)
@@ -519,24 +517,24 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     const uint32_t half = L >> 6;
     const uint32_t hl = L & 63u;
     const uint32_t lane_off = (warp * 32u) << 16;
-    const uint32_t pairw = warp & 1u;                  // warps 0,2 -> pair 0; 1,3 -> pair 1
     const uint32_t partner = L ^ 64u;
     uint32_t qn = 0, pb = 0, nx = 0, qd = 0;
     uint32_t s_i = 0, s_u = 0;                         // logits buffer, and its use count
     bool ok = true;
     // one float from the partner lane (the other half of the same head)
+    // Each lane owns two 64-bit slots (alternating exchanges) and stores (exchange number, value)
+    // in one word; the partner polls for the number it expects. A lane can reuse a slot only
+    // after the partner has answered the next exchange, so no unread value is overwritten.
     auto swap_partner = [&](float mine) -> float {
-      const uint32_t par = nx & 1u, ph = (nx >> 1) & 1u;
-      ++nx;
-      xmax[par * 128 + L] = mine;
-      __syncwarp();
-      uint32_t got = 1;
-      if (lane == 0) {
-        mbar_arrive(pair_bar(pairw, par));
-        got = wt.wait(pair_bar(pairw, par), ph, 37) ? 1u : 0u;
-      }
-      if (!__shfl_sync(0xffffffffu, got, 0)) ok = false;
-      return xmax[par * 128 + partner];
+      const uint32_t par = nx & 1u;
+      const uint32_t tag = ++nx;
+      const uint64_t word = (static_cast<uint64_t>(tag) << 32) | __float_as_uint(mine);
+      asm volatile("st.volatile.shared.u64 [%0], %1;" ::"r"(sbase + C::OFF_XMAX + (par * 128u + L) * 8u), "l"(word)
+                   : "memory");
+      uint32_t v = 0;
+      const bool okl = wt.wait_tagged(sbase + C::OFF_XMAX + (par * 128u + partner) * 8u, tag, 37, v);
+      if (!__all_sync(0xffffffffu, okl)) ok = false;
+      return __uint_as_float(v);
     };
     for (int32_t qi = cid; qi < p.n_queries && ok; qi += ncl, ++qn) {
       const uint32_t slot = qn & 1u, sph = (qn >> 1) & 1u;
