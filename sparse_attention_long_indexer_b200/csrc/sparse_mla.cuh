@@ -27,7 +27,7 @@
 //    stages; two groups of four producer warps run the two rings independently.
 //  * softmax: one thread per TMEM lane holds half a row (32 logits); the two halves of a row
 //    exchange their maxima through shared memory; online softmax in the log2 domain, the
-//    output rescaled only when the running max grows by more than 8 (exact: the final
+//    output rescaled only when the running max grows by more than 32 (exact: the final
 //    normalisation uses the same max). P is announced with a CTA-scope arrive; the odd CTA's
 //    announcements reach the even CTA through one relay thread.
 //  * two issuing threads share the tensor pipe: one for the logits MMAs, one for the output
@@ -49,6 +49,14 @@ constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kBlk = 64;                 // selected rows per block
 constexpr int kMaxTopk = 2048;
+// The running max m2 (log2 domain) is raised, and O rescaled, only when a block's max exceeds it
+// by more than this. Until then P = 2^(z - m2) <= 2^32: bf16 P and the fp32 O and row sum have
+// the exponent range of fp32, so nothing overflows unless |kv| > 2^80, and the final
+// normalisation divides by the row sum taken against the same m2, so the result is unchanged.
+// A rescale waits for the previous block's output MMAs, a stall of the whole pipeline, so it
+// should be rare: with a bound of 8, random logits with a spread of several units trigger it in
+// a sizeable fraction of blocks for some warp.
+constexpr float kLazyRescale = 32.0f;
 
 struct AttnCfg {
   static constexpr int SB_STAGES = 3;                    // own rows, all dims (logits operand)
@@ -590,7 +598,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         float mb = mraw * sc;
         mb = fmaxf(mb, swap_partner(mb));
         if (!ok) break;
-        const bool need = (mb > m2 + 8.0f);
+        const bool need = (mb > m2 + kLazyRescale);
         float alpha = 1.0f;
         if (need) {
           alpha = (m2 == -INFINITY) ? 0.0f : ex2_approx(m2 - mb);
