@@ -36,7 +36,7 @@ constexpr int kIdxHeads = 64;     // H_I (padded)
 constexpr int kIdxDim = 128;      // d_I (padded), one 128-byte row per head / key
 constexpr int kKeyTile = 128;     // keys per MMA tile (M)
 constexpr int kDecodeChunk = 8192;  // keys per decode work item
-constexpr int kSyncTiles = 2;       // key tiles between two capacity checks of a candidate buffer
+constexpr int kSyncTiles = 4;       // key tiles between two capacity checks of a candidate buffer
 
 template <int NQ>
 struct IdxCfg {
@@ -326,6 +326,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         q_strict[q] = 0;
       }
       named_barrier(bar_id, C::GROUP_THREADS);
+      // the query's admission threshold, changed only by a capacity check; kept in registers
+      uint32_t thr_r = 0, strict_r = 0;
       const int32_t qpos = q_valid ? it.len - p.n_q + i : -1;
       const float4* w4 = reinterpret_cast<const float4*>(wq + q * kIdxHeads);
       // with few epilogue warps the query's head weights stay in registers for the whole item
@@ -342,6 +344,11 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         return __ldg(ks_row + min(s_lane + t * kKeyTile, it.s_end - 1));
       };
       float ks_next = key_scale(0);
+      // Candidates are appended at the capacity checks, not per tile: bit j of pbits says that
+      // this lane's key of the tile j tiles back passed, pk[j] is its score key. A check thus
+      // takes one atomic per warp for up to kSyncTiles tiles.
+      uint32_t pk[kSyncTiles];
+      uint32_t pbits = 0;
       for (int32_t t = 0; t < it.ntiles; ++t, ++g) {
         const uint32_t buf = g % C::NBUF, acc_ph = (g / C::NBUF) & 1u;
         const int32_t s = s_lane + t * kKeyTile;
@@ -350,6 +357,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         ks_next = key_scale(t + 1);
         // every lane waits (no divergent branch); the warp then runs the collective TMEM loads
         const bool ok = __all_sync(0xffffffffu, wt.wait(acc_full(buf, half), acc_ph, 8)) != 0;
+        bool pass = false;
+        uint32_t key = 0;
         if (ok) {
           tc_fence_after();
           const uint32_t col = buf * C::N + q * kIdxHeads;
@@ -400,25 +409,42 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
           }
           const float score =
               (((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y))) * ks;
-          const uint32_t key = score_key(score);
+          key = score_key(score);
           const bool valid = in_range && s <= qpos;
-          const uint32_t thr = q_thr[q];
-          const bool pass = valid && (key > thr || (key == thr && q_strict[q] == 0));
-          const uint32_t m = __ballot_sync(0xffffffffu, pass);
-          if (m) {
-            uint32_t base = 0;
-            if (lane == 0) base = atomicAdd(&q_count[q], __popc(m));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (pass) {
-              const uint32_t at = base + __popc(m & ((1u << lane) - 1u));
-              cq_keys[at] = key;
-              cq_pos[at] = s;
-            }
-          }
+          pass = valid && (key > thr_r || (key == thr_r && strict_r == 0));
         }
+#pragma unroll
+        for (int j = kSyncTiles - 1; j > 0; --j) pk[j] = pk[j - 1];
+        pk[0] = key;
+        pbits = (pbits << 1) | (pass ? 1u : 0u);
         // capacity check every kSyncTiles tiles: between two checks at most kSyncTiles * 128
         // candidates arrive, and a check leaves at most CAND - kSyncTiles * 128
         if (t % kSyncTiles != kSyncTiles - 1 && t + 1 != it.ntiles) continue;
+        {
+          // append this warp's passes of the tiles since the last check (tile t - j for bit j)
+          const uint32_t lt = (1u << lane) - 1u;
+          uint32_t off[kSyncTiles];
+          uint32_t total = 0;
+#pragma unroll
+          for (int j = 0; j < kSyncTiles; ++j) {
+            const uint32_t mj = __ballot_sync(0xffffffffu, (pbits >> j) & 1u);
+            off[j] = total + __popc(mj & lt);
+            total += __popc(mj);
+          }
+          if (total) {
+            uint32_t base = 0;
+            if (lane == 0) base = atomicAdd(&q_count[q], total);
+            base = __shfl_sync(0xffffffffu, base, 0);
+#pragma unroll
+            for (int j = 0; j < kSyncTiles; ++j) {
+              if ((pbits >> j) & 1u) {
+                cq_keys[base + off[j]] = pk[j];
+                cq_pos[base + off[j]] = s - j * kKeyTile;
+              }
+            }
+          }
+          pbits = 0;
+        }
         if (uniform_stop()) { stop = true; break; }
         const uint32_t n = q_count[q];
         if (n > static_cast<uint32_t>(C::CAND - kSyncTiles * kKeyTile)) {
@@ -442,6 +468,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
             q_strict[q] = 0;
           }
           named_barrier(bar_id, C::GROUP_THREADS);
+          thr_r = q_thr[q];
+          strict_r = q_strict[q];
         }
       }
       if (stop) break;
