@@ -96,6 +96,7 @@ struct AttnCfg {
   static_assert(SB_BYTES % 1024 == 0 && Q_TMEM_DIMS / 2 + COL_Q <= TMEM_COLS, "layout");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(P_BUFS == 1 || P_BUFS == 2, "P buffers");
+  static_assert(SB_STAGES <= 4 && VR_STAGES <= 4 && S_BUFS <= 3, "barrier slots");
 };
 
 struct AttnParams {
@@ -154,16 +155,17 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
   // local barriers (both CTAs)
   auto info_full = [&](int i) { return B(0 + i); };
   auto info_empty = [&](int i) { return B(2 + i); };
-  auto sb_empty = [&](int s) { return B(4 + s); };       // commit: logits operand stage consumed
-  auto vr_empty = [&](int s) { return B(7 + s); };       // commit: output operand stage consumed
+  // ring barriers: stages 0..2 / 0..1 in their first slots, further stages in free slots
+  auto sb_empty = [&](int s) { return s < 3 ? B(4 + s) : B(15); };         // commit: logits stage consumed
+  auto vr_empty = [&](int s) { return s < 2 ? B(7 + s) : B(12 + (s - 2)); };  // commit: output stage consumed
   const uint32_t q_tma = B(9);                           // this CTA's smem part of q landed (TMA)
   const uint32_t q_empty = B(10);                        // commit: all logits MMAs of a query done
   auto s_full = [&](uint32_t i) { return B(31 + i); };   // commit: logits buffer i ready (3)
   auto p_empty = [&](uint32_t j) { return B(34 + j); };  // commit: output MMA that read P buffer j done (2)
   const uint32_t o_full = B(14);                         // commit: all output MMAs of a query done
   // barriers of the even CTA, arrived on by both CTAs
-  auto sb_full2 = [&](int s) { return B(19 + s); };
-  auto vr_full2 = [&](int s) { return B(22 + s); };
+  auto sb_full2 = [&](int s) { return s < 3 ? B(19 + s) : B(16); };
+  auto vr_full2 = [&](int s) { return s < 2 ? B(22 + s) : B(25 + (s - 2)); };
   const uint32_t q_full2 = B(24);
   // logits buffer i free again: arrived by the output-MMA thread once it has seen the P of the
   // block that used the buffer (the softmax reads the logits before it writes P)
@@ -188,6 +190,8 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
       mbar_init(info_full(i), 1);
       // softmax warps + output-ring producer warps (+ the MMA thread in the even CTA)
       mbar_init(info_empty(i), C::SOFTMAX_WARPS + C::GROUP_WARPS + (leader ? 2 : 1));
+    }
+    for (int i = 0; i < C::VR_STAGES; ++i) {
       mbar_init(vr_empty(i), 1);
       mbar_init(vr_full2(i), 2 * C::GROUP_WARPS);
     }
