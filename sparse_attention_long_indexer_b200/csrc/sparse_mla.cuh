@@ -21,12 +21,14 @@
 //    dims with CTA r supplying dims 256i + 128r .. +127. Each CTA accumulates all 512 dims of
 //    its 64 heads (TMEM: 256 columns; lane m / 64+m hold the low / high 128 dims of each
 //    instruction).
-//  * per 64-row block, CTA r gathers its 32 rows completely (logits operand, a 2-stage ring
+//  * per 64-row block, CTA r gathers its 32 rows completely (logits operand, a 3-stage ring
 //    freed by the logits MMA) and all 64 rows' dims it supplies to the output product (a
 //    2-stage ring freed by the output MMA), with 16-byte cp.async into 128-byte-swizzled
-//    stages; two groups of four producer warps run the two rings independently.
+//    stages; two groups of four producer warps run the two rings independently. Rows are
+//    read straight from the query's index row, one block ahead; padding and out-of-range
+//    entries are gathered as zero rows and masked in the softmax.
 //  * softmax: one thread per TMEM lane holds half a row (32 logits); the two halves of a row
-//    exchange their maxima through shared memory; online softmax in the log2 domain, the
+//    exchange their maxima through tagged 64-bit shared-memory words; online softmax in the log2 domain, the
 //    output rescaled only when the running max grows by more than 32 (exact: the final
 //    normalisation uses the same max). P is announced with a CTA-scope arrive; the odd CTA's
 //    announcements reach the even CTA through one relay thread.
