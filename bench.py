@@ -34,6 +34,12 @@ import synthetic  # noqa: E402
 
 METRIC = "DSA prefill query-tokens/s (indexer+top-k+sparse MLA) at 128K ctx, k=2048"
 UNIT = "query-tokens/s"
+DECODE_METRIC = "DSA decode sequences/s (indexer+top-k+sparse MLA), 64 sequences, len ~ U[4K,128K], k=2048"
+DECODE_UNIT = "sequences/s"
+
+
+def _metric(cfg):
+    return (DECODE_METRIC, DECODE_UNIT) if cfg.is_decode else (METRIC, UNIT)
 
 
 def _peaks():
@@ -45,16 +51,30 @@ def _peaks():
     return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
-def _work(cfg):
-    """Algorithmic work per launch of each stage (causal prefill, B sequences of length L)."""
-    L, B = cfg.max_len, cfg.batch
-    pairs = B * L * (L + 1) // 2                              # causal (t, s) pairs, s <= t
-    k = min(cfg.topk, L)
-    sel_rows = B * (k * (k + 1) // 2 + (L - k) * cfg.topk)  # sum over t of min(k, t+1)
+def _work(cfg, seed=0):
+    """Algorithmic work per launch of each stage.
+
+    Prefill: B causal sequences of length L. Decode: one query per sequence at position
+    len_b - 1 over its len_b cached keys (lengths from the seeded generator). The byte counts
+    are the compulsory HBM traffic: every input read once, every output written once."""
+    B, k = cfg.batch, cfg.topk
+    if cfg.is_decode:
+        lens = [int(x) for x in synthetic.lengths(cfg, seed)]
+        pairs = sum(lens)
+        sel_rows = sum(min(k, n) for n in lens)
+    else:
+        L = cfg.max_len
+        pairs = B * L * (L + 1) // 2                              # causal (t, s) pairs, s <= t
+        kk = min(k, L)
+        sel_rows = B * (kk * (kk + 1) // 2 + (L - kk) * k)        # sum over t of min(k, t+1)
+    n_tok = B * cfg.n_q
+    keys = pairs if cfg.is_decode else B * cfg.max_len            # keys read once per launch
     return {
         "indexer_flop": pairs * 2 * cfg.n_idx_heads * cfg.idx_dim,                     # FP8 MACs x 2
         "attn_flop": sel_rows * 2 * cfg.n_heads * (cfg.d_qk + cfg.d_v),                 # QK^T + PV
         "attn_gather_bytes": sel_rows * cfg.d_qk * 2,
+        "indexer_bytes": keys * (cfg.idx_dim + 4) + n_tok * (cfg.n_idx_heads * (cfg.idx_dim + 2) + 4 + k * 4),
+        "attn_bytes": sel_rows * cfg.d_qk * 2 + n_tok * (cfg.n_heads * ((cfg.d_qk + cfg.d_v) * 2 + 4) + k * 4),
         "pairs": pairs, "sel_rows": sel_rows,
     }
 
@@ -152,6 +172,53 @@ def _oracle_rows(cfg, seed, rows, cache=None):
 def _shuffled_rows(cfg, n, seed):
     rows = synthetic.sample_rows(cfg.n_q, n, seed)
     return [rows[i] for i in np.random.default_rng(seed).permutation(len(rows))]
+
+
+def _oracle_decode(cfg, seed, seqs):
+    """Runs the fp64 oracle (full path) on the decode queries of the listed sequences.
+
+    Each sequence's caches (its len_b keys and latent rows) are regenerated first; only the
+    oracle itself is timed. Returns (oracle seconds, BLAS threads)."""
+    import oracle
+    from tests.dsa_cases import u16
+    lens = synthetic.lengths(cfg, seed)
+    spent, threads = 0.0, 1
+    for b in seqs:
+        n = int(lens[b])
+        kc, ks = synthetic.gen_k_idx(cfg, seed, b=b, s_range=range(0, n))
+        kv = u16(synthetic.gen_kv(cfg, seed, b=b, positions=range(0, n)))
+        qc, qs = synthetic.gen_q_idx(cfg, seed, tokens=[b * cfg.n_q])
+        w = synthetic.gen_w(cfg, seed, tokens=[b * cfg.n_q])
+        q = synthetic.gen_q(cfg, seed, tokens=[b * cfg.n_q])
+        t0 = time.perf_counter()
+        oracle.dsa_row(qc[0].numpy(), float(qs[0]), u16(w[0]), kc.numpy(), ks.numpy(), u16(q[0]), kv, n - 1,
+                       cfg.topk, cfg.d_v, cfg.softmax_scale)
+        spent += time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        pass
+    return spent, threads
+
+
+def cpu_baseline_decode(cfg, seed, budget_s=20.0):
+    order = [int(i) for i in np.random.default_rng(seed + 99).permutation(cfg.batch)]
+    t_start = time.perf_counter()
+    done, spent, threads = 0, 0.0, 1
+    for b in order:
+        # cache regeneration (about 3 s per sequence on the host) dominates the wall time, so the
+        # sample also stops after twice the oracle budget of wall time
+        if spent >= budget_s or (done > 0 and time.perf_counter() - t_start >= 2 * budget_s):
+            break
+        dt, threads = _oracle_decode(cfg, seed, [b])
+        spent += dt
+        done += 1
+    return {"value": done / spent, "unit": DECODE_UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{done} seeded random sequences of the decode workload (full path per sequence: fp64 index "
+                      f"scores over its len_b cached keys, stable sort, fp64 attention over the k selected rows); "
+                      f"{spent:.1f} s of oracle time, {time.perf_counter() - t_start:.1f} s wall incl. cache "
+                      f"regeneration"}
 
 
 def cpu_baseline(cfg, seed, budget_s=20.0):
@@ -264,7 +331,9 @@ def run_ours(args, cfg, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world)
-    return dict(total_ms=total_ms, idx_ms=idx_ms, att_ms=att_ms, clocks=clocks, e2e=e2e)
+    # kernels per step: the indexer is one launch (decode: chunk kernel + merge), the attention one
+    launches = (2 if cfg.is_decode else 1) * int(do_idx) + int(do_att)
+    return dict(total_ms=total_ms, idx_ms=idx_ms, att_ms=att_ms, clocks=clocks, e2e=e2e, launches_per_step=launches)
 
 
 
@@ -320,6 +389,62 @@ def run_e2e_whole(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
             "pinned": pinned}
 
 
+def run_e2e_decode(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
+    """A decode step end to end through the public API, as a serving loop runs it: the caches
+    (indexer keys, their scales and the latent rows) stay resident on the device; every step
+    uploads the new queries' inputs and the lengths from pinned host memory and reads back out,
+    lse and idx. Appending the new token's own cache rows belongs to the caller's cache
+    management and is not part of this path."""
+    B = cfg.batch
+    q_side = ["q_idx", "w", "q", "lengths"]
+    try:
+        host = {n: torch.empty(g[n].shape, dtype=g[n].dtype, pin_memory=True) for n in q_side}
+        host_qs = torch.empty((B * cfg.n_q,), dtype=torch.float32, pin_memory=True)
+        host_out = torch.empty((B, cfg.n_q, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, pin_memory=True)
+        host_lse = torch.empty((B, cfg.n_q, cfg.n_heads), dtype=torch.float32, pin_memory=True)
+        host_idx = torch.empty((B, cfg.n_q, cfg.topk), dtype=torch.int32, pin_memory=True)
+    except RuntimeError:
+        return {"value": None, "unit": DECODE_UNIT, "note": "pinned host allocation failed"}
+    for n in q_side:
+        host[n].copy_(g[n])
+    host_qs.copy_(scales[:B * cfg.n_q])
+    dev_in = {n: torch.empty_like(g[n]) for n in q_side}
+    dev_scales = scales.clone()                      # key scales resident; query scales rewritten per step
+    out = torch.empty(host_out.shape, dtype=host_out.dtype, device=dev)
+    lse = torch.empty(host_lse.shape, dtype=host_lse.dtype, device=dev)
+    idx = torch.empty(host_idx.shape, dtype=host_idx.dtype, device=dev)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in q_side) + host_qs.numel() * 4
+    d2h = host_out.numel() * 2 + host_lse.numel() * 4 + host_idx.numel() * 4
+
+    def step():
+        for n in q_side:
+            dev_in[n].copy_(host[n], non_blocking=True)
+        dev_scales[:B * cfg.n_q].copy_(host_qs, non_blocking=True)
+        dsa.dsa_forward(dims, dev_in["q_idx"], dev_in["w"], g["k_idx"], dev_scales, dev_in["lengths"], cfg.topk,
+                        dev_in["q"], g["kv"], idx, out, lse, ws.buf, stream)
+        host_out.copy_(out, non_blocking=True)
+        host_lse.copy_(lse, non_blocking=True)
+        host_idx.copy_(idx, non_blocking=True)
+
+    steps = max(3, args.steps)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(a.elapsed_time(b), dev)
+    ws.check()
+    return {"value": aggregate_value(B * cfg.n_q, steps, world, ms), "unit": DECODE_UNIT, "steps": steps,
+            "ms_per_step": ms / steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "pinned": True,
+            "caches": "resident on the device (uploaded once, outside the timed region)"}
+
+
 def run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
     """The step end to end through the public API: inputs from pinned host memory, results read back.
 
@@ -330,6 +455,8 @@ def run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
     n_q = i1 - i0 and lengths = i1, the query positions the header defines; it computes exactly what
     the whole call computes for those queries.
     """
+    if cfg.is_decode:
+        return run_e2e_decode(args, cfg, dsa, dims, g, scales, ws, dev, stream, world)
     if cfg.batch != 1 or args.e2e_chunk <= 0:
         return run_e2e_whole(args, cfg, dsa, dims, g, scales, ws, dev, stream, world)
     L, H, dv, k = cfg.max_len, cfg.n_heads, cfg.d_v, cfg.topk
@@ -439,9 +566,10 @@ def run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 10; decode: 1000, so clocks are sampled during the timed region)")
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="prefill_128k", choices=["prefill_4k", "prefill_32k", "prefill_128k"])
+    ap.add_argument("--workload", default="prefill_128k", choices=["prefill_4k", "prefill_32k", "prefill_128k", "decode"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=2)
@@ -457,6 +585,8 @@ def main():
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     cfg = synthetic.config(args.workload)
+    if args.steps is None:
+        args.steps = 1000 if cfg.is_decode and args.impl == "ours" else 10
     if args.seq_len:
         import dataclasses
         cfg = dataclasses.replace(cfg, n_q=args.seq_len, max_len=args.seq_len, name=f"prefill_L{args.seq_len}",
@@ -489,74 +619,117 @@ def main():
 
 def report(args, cfg, res, world):
     peaks = _peaks()
-    w = _work(cfg)
+    w = _work(cfg, rank_seed(args.seed, 0))
+    metric, unit = _metric(cfg)
     ms_step = res["total_ms"] / args.steps
     idx_ms = statistics.mean(res["idx_ms"])
     att_ms = statistics.mean(res["att_ms"])
     fp8_peak = 2.0 * peaks["bf16_sustained"]          # nominal fp8:bf16 ratio 2 (4.5 : 2.25 PF)
     stages = {}
-    if args.stage in ("all", "indexer"):
-        stages["indexer_topk"] = {"ms": idx_ms, "bound": "tensor",
-                                  "achieved": w["indexer_flop"] / (idx_ms / 1e3) / 1e12, "peak": fp8_peak,
-                                  "unit": "TFLOP/s",
-                                  "peak_note": f"fp8 = 2 x {peaks['source']} sustained bf16 {peaks['bf16_sustained']}"}
-    if args.stage in ("all", "attention"):
-        stages["sparse_mla_attn"] = {"ms": att_ms, "bound": "tensor",
-                                     "achieved": w["attn_flop"] / (att_ms / 1e3) / 1e12,
-                                     "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                                     "peak_note": f"{peaks['source']} sustained bf16",
-                                     "gather_GBps": w["attn_gather_bytes"] / (att_ms / 1e3) / 1e9}
-    for k, s in stages.items():
-        s["frac"] = s["achieved"] / s["peak"]
+    if cfg.is_decode:
+        # one query per sequence: both stages stream their inputs once, so HBM bounds them
+        hbm = {"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_note": f"{peaks['source']} HBM copy"}
+        if args.stage in ("all", "indexer"):
+            stages["indexer_topk"] = dict(hbm, ms=idx_ms, us=idx_ms * 1e3,
+                                          achieved=w["indexer_bytes"] / (idx_ms / 1e3) / 1e9,
+                                          bytes=w["indexer_bytes"],
+                                          tflops_fp8=w["indexer_flop"] / (idx_ms / 1e3) / 1e12)
+        if args.stage in ("all", "attention"):
+            stages["sparse_mla_attn"] = dict(hbm, ms=att_ms, us=att_ms * 1e3,
+                                             achieved=w["attn_bytes"] / (att_ms / 1e3) / 1e9,
+                                             bytes=w["attn_bytes"],
+                                             tflops_bf16=w["attn_flop"] / (att_ms / 1e3) / 1e12)
+    else:
+        if args.stage in ("all", "indexer"):
+            stages["indexer_topk"] = {"ms": idx_ms, "bound": "tensor",
+                                      "achieved": w["indexer_flop"] / (idx_ms / 1e3) / 1e12, "peak": fp8_peak,
+                                      "unit": "TFLOP/s",
+                                      "peak_note": f"fp8 = 2 x {peaks['source']} sustained bf16 "
+                                                   f"{peaks['bf16_sustained']}"}
+        if args.stage in ("all", "attention"):
+            stages["sparse_mla_attn"] = {"ms": att_ms, "bound": "tensor",
+                                         "achieved": w["attn_flop"] / (att_ms / 1e3) / 1e12,
+                                         "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                                         "peak_note": f"{peaks['source']} sustained bf16",
+                                         "gather_GBps": w["attn_gather_bytes"] / (att_ms / 1e3) / 1e9}
+    for k, st in stages.items():
+        st["frac"] = st["achieved"] / st["peak"]
     dom = max(stages, key=lambda k: stages[k]["ms"])
     ds = stages[dom]
     roofline = {"kernel": dom, "bound": ds["bound"], "achieved": ds["achieved"], "peak": ds["peak"],
                 "unit": ds["unit"], "frac": ds["frac"],
                 "traffic": _traffic("indexer" if dom == "indexer_topk" else "attention", cfg.name)}
+    if cfg.is_decode:
+        lo, hi = cfg.len_range
+        conf = {"workload": f"{cfg.description}; H_I={cfg.n_idx_heads} d_I={cfg.idx_dim} FP8 e4m3, "
+                            f"H={cfg.n_heads}, d_qk={cfg.d_qk}, d_v={cfg.d_v}, bf16",
+                "global_batch": cfg.batch * world, "seq_len": cfg.max_len, "lengths": f"U[{lo},{hi}] (seeded)",
+                "topk": cfg.topk,
+                "parallelism": f"{world} x {cfg.batch} independent sequences, one group per GPU (no data-path "
+                               f"collective)",
+                "l2": "caches larger than L2 (latent rows alone are %.1f GB)"
+                      % (cfg.batch * cfg.max_len * cfg.d_qk * 2 / 1e9)}
+    else:
+        conf = {"workload": f"{cfg.name}: {cfg.description}; H_I={cfg.n_idx_heads} d_I={cfg.idx_dim} FP8 e4m3, "
+                            f"H={cfg.n_heads}, d_qk={cfg.d_qk}, d_v={cfg.d_v}, bf16",
+                "global_batch": cfg.batch * world, "seq_len": cfg.max_len, "topk": cfg.topk,
+                "parallelism": f"{world} independent sequences, one per GPU (no data-path collective)",
+                "l2": "inputs larger than L2 (q alone is %.1f GB)" % (cfg.n_q * cfg.n_heads * cfg.d_qk * 2 / 1e9)}
     line = {
-        "metric": METRIC, "value": aggregate_value(cfg.batch * cfg.n_q, args.steps, world, res["total_ms"]),
-        "unit": UNIT,
+        "metric": metric, "value": aggregate_value(cfg.batch * cfg.n_q, args.steps, world, res["total_ms"]),
+        "unit": unit,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3+bf16 (fp32 accumulate)",
-        "data": "synthetic",
-        "config": {"workload": f"{cfg.name}: {cfg.description}; H_I={cfg.n_idx_heads} d_I={cfg.idx_dim} FP8 e4m3, "
-                               f"H={cfg.n_heads}, d_qk={cfg.d_qk}, d_v={cfg.d_v}, bf16",
-                   "global_batch": cfg.batch * world, "seq_len": cfg.max_len, "topk": cfg.topk,
-                   "parallelism": f"{world} independent sequences, one per GPU (no data-path collective)",
-                   "l2": "inputs larger than L2 (q alone is %.1f GB)" % (cfg.n_q * cfg.n_heads * cfg.d_qk * 2 / 1e9)},
+        "data": "synthetic", "config": conf,
         "roofline": roofline, "stages": stages,
-        "gpu_launches": len(stages) * args.steps,
+        "gpu_launches": res.get("launches_per_step", len(stages)) * args.steps,
         "clocks": res["clocks"], "e2e": res["e2e"],
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, args.seed, args.cpu_budget)
+        line["cpu_baseline"] = (cpu_baseline_decode if cfg.is_decode else cpu_baseline)(cfg, args.seed,
+                                                                                         args.cpu_budget)
     return line
 
 
 def run_reference(args, cfg, world):
     """The fp64 oracle as the reference arm: each step is a bounded sample of the workload."""
-    rows_all = _shuffled_rows(cfg, 100000, args.seed + 7)
-    per_step = 4
-    cache = None
-    pos = 0
-    for _ in range(args.warmup):
-        _, _, cache = _oracle_rows(cfg, args.seed, rows_all[pos:pos + per_step], cache)
-        pos += per_step
+    metric, unit = _metric(cfg)
     total, threads = 0.0, 1
-    for _ in range(args.steps):
-        dt, threads, cache = _oracle_rows(cfg, args.seed, rows_all[pos:pos + per_step], cache)
-        total += dt
-        pos += per_step
+    if cfg.is_decode:
+        order = [int(i) for i in np.random.default_rng(args.seed + 7).permutation(cfg.batch)]
+        per_step = 1
+        pos = 0
+        for _ in range(args.warmup):
+            _oracle_decode(cfg, args.seed, order[pos % cfg.batch:pos % cfg.batch + 1])
+            pos += 1
+        for _ in range(args.steps):
+            dt, threads = _oracle_decode(cfg, args.seed, order[pos % cfg.batch:pos % cfg.batch + 1])
+            total += dt
+            pos += 1
+        sample = (f"{per_step} seeded random sequence per step of the {cfg.name} workload, full path (fp64 index "
+                  f"scores over its cached keys, stable sort, fp64 attention)")
+    else:
+        rows_all = _shuffled_rows(cfg, 100000, args.seed + 7)
+        per_step = 4
+        cache = None
+        pos = 0
+        for _ in range(args.warmup):
+            _, _, cache = _oracle_rows(cfg, args.seed, rows_all[pos:pos + per_step], cache)
+            pos += per_step
+        for _ in range(args.steps):
+            dt, threads, cache = _oracle_rows(cfg, args.seed, rows_all[pos:pos + per_step], cache)
+            total += dt
+            pos += per_step
+        sample = (f"{per_step} seeded uniformly-random query rows per step of the {cfg.name} workload, full path "
+                  f"per row (fp64 index scores, stable sort, fp64 attention)")
     value = per_step * args.steps / total
-    sample = (f"{per_step} seeded uniformly-random query rows per step of the {cfg.name} workload, full path per "
-              f"row (fp64 index scores, stable sort, fp64 attention)")
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": f"{cfg.name}: {cfg.description}", "global_batch": cfg.batch,
                        "seq_len": cfg.max_len, "topk": cfg.topk, "parallelism": "CPU oracle, rank 0 only"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
-            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -1,0 +1,60 @@
+"""Host logic of the benchmark's report (no GPU): algorithmic work and the JSON line's shape for
+the prefill and decode workloads."""
+import types
+
+import pytest
+
+import bench
+import synthetic
+
+
+def _args(**kw):
+    d = dict(seed=0, steps=10, warmup=3, stage="all", no_cpu_baseline=True, cpu_budget=1.0)
+    d.update(kw)
+    return types.SimpleNamespace(**d)
+
+
+def _res(launches):
+    return dict(total_ms=20.0, idx_ms=[1.2] * 10, att_ms=[0.8] * 10, clocks=None, e2e=None,
+                launches_per_step=launches)
+
+
+def test_decode_work_follows_the_seeded_lengths():
+    cfg = synthetic.config("decode")
+    lens = [int(x) for x in synthetic.lengths(cfg, 0)]
+    w = bench._work(cfg, 0)
+    # the decode query sits at position len-1 and scores every cached key 0..len-1
+    assert w["pairs"] == sum(lens)
+    assert w["sel_rows"] == sum(min(cfg.topk, n) for n in lens)
+    assert w["indexer_flop"] == sum(lens) * 2 * 64 * 128
+    # keys are read once: 128 code bytes and a 4-byte scale each, plus the query side and idx
+    assert w["indexer_bytes"] == sum(lens) * 132 + cfg.batch * (64 * 130 + 4 + cfg.topk * 4)
+    assert w["attn_bytes"] == w["sel_rows"] * 1152 + cfg.batch * (128 * (1088 * 2 + 4) + cfg.topk * 4)
+
+
+def test_prefill_work_is_the_causal_count():
+    cfg = synthetic.config("prefill_4k")
+    w = bench._work(cfg, 0)
+    L, k = 4096, 2048
+    assert w["pairs"] == L * (L + 1) // 2
+    assert w["sel_rows"] == k * (k + 1) // 2 + (L - k) * k
+
+
+def test_decode_line_is_hbm_bound_in_sequences_per_second():
+    cfg = synthetic.config("decode")
+    line = bench.report(_args(), cfg, _res(3), 1)
+    assert line["unit"] == "sequences/s" and line["metric"].startswith("DSA decode")
+    assert line["value"] == pytest.approx(64 * 10 / 0.020)
+    assert line["gpu_launches"] == 30
+    for st in line["stages"].values():
+        assert st["bound"] == "hbm" and st["unit"] == "GB/s"
+        assert st["frac"] == pytest.approx(st["achieved"] / st["peak"])
+    assert line["roofline"]["kernel"] == "indexer_topk"
+
+
+def test_prefill_line_keeps_the_headline_metric():
+    cfg = synthetic.config("prefill_128k")
+    line = bench.report(_args(), cfg, _res(2), 1)
+    assert line["metric"] == bench.METRIC and line["unit"] == "query-tokens/s"
+    assert line["stages"]["indexer_topk"]["bound"] == "tensor"
+    assert line["gpu_launches"] == 20
