@@ -256,7 +256,7 @@ dsa_status run_indexer(const dsa_dims& d, const uint8_t* q_idx, const __nv_bfloa
     if (!encode_rows_u8(&map_q, q_idx, static_cast<uint64_t>(kIdxHeads), static_cast<uint64_t>(d.batch),
                         kIdxHeads))
       return DSA_ERR_CUDA;
-    const int grid = std::min(p.n_items, dev.sms);
+    const int grid = std::min(p.n_items, IdxCfg<1>::CTAS_PER_SM * dev.sms);
     indexer_topk_kernel<1><<<grid, IdxCfg<1>::THREADS, IdxCfg<1>::SMEM_BYTES, st>>>(map_q, map_k, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return DSA_ERR_CUDA;
@@ -556,7 +556,7 @@ extern "C" dsa_status dsa_indexer_topk_decode_noalloc(const dsa_dims* dims, cons
   if (!encode_rows_u8(&map_k, k_idx, static_cast<uint64_t>(d.max_len), static_cast<uint64_t>(d.batch), kKeyTile) ||
       !encode_rows_u8(&map_q, q_idx, static_cast<uint64_t>(kIdxHeads), static_cast<uint64_t>(d.batch), kIdxHeads))
     return DSA_ERR_CUDA;
-  const int grid = std::min(p.n_items, dev.sms);
+  const int grid = std::min(p.n_items, IdxCfg<1>::CTAS_PER_SM * dev.sms);
   indexer_topk_kernel<1><<<grid, IdxCfg<1>::THREADS, IdxCfg<1>::SMEM_BYTES, st>>>(map_q, map_k, p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   MergeParams mp{p.part_keys, p.part_pos, p.part_count, out_idx, n_chunks, topk};

@@ -53,7 +53,9 @@ struct IdxCfg {
   static constexpr int PRODUCER_WARP = EPI_WARPS;
   static constexpr int MMA_WARP = EPI_WARPS + 1;
   static constexpr int THREADS = (EPI_WARPS + 2) * 32;
-  static constexpr int STAGES = (NQ == 4) ? 4 : (NQ == 2) ? 6 : 8;
+  static constexpr int STAGES = (NQ == 4) ? 4 : (NQ == 2) ? 6 : 4;
+  // decode (one query per item) runs two CTAs per SM, so that two items' epilogues share an SM
+  static constexpr int CTAS_PER_SM = (NQ == 1) ? 2 : 1;
   static constexpr int Q_BYTES = NQ * kIdxHeads * kIdxDim;
   static constexpr int K_BYTES = kKeyTile * kIdxDim;       // 16 KB
   static constexpr int TMEM_COLS = NBUF * N;
@@ -144,7 +146,7 @@ __device__ __forceinline__ int32_t item_of(int32_t round, int32_t cta, int32_t G
 }
 
 template <int NQ>
-__global__ void __launch_bounds__(IdxCfg<NQ>::THREADS, 1)
+__global__ void __launch_bounds__(IdxCfg<NQ>::THREADS, IdxCfg<NQ>::CTAS_PER_SM)
 indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                     const IndexerParams p) {
   using C = IdxCfg<NQ>;
@@ -521,7 +523,8 @@ template <int T>
 __global__ void __launch_bounds__(T) merge_partials_kernel(const MergeParams p) {
   __shared__ SelectScratch sc;
   __shared__ uint32_t s_count[1024 + 1];
-  const uint32_t tid = threadIdx.x;
+  __shared__ uint32_t s_lo[T / 32], s_hi[T / 32];
+  const uint32_t tid = threadIdx.x, lane = tid & 31u;
   const int32_t b = blockIdx.x;
   const size_t base_slot = static_cast<size_t>(b) * p.n_chunks;
   for (int32_t c = tid; c < p.n_chunks; c += T) s_count[c] = static_cast<uint32_t>(p.part_count[base_slot + c]);
@@ -530,60 +533,106 @@ __global__ void __launch_bounds__(T) merge_partials_kernel(const MergeParams p) 
   for (int32_t c = 0; c < p.n_chunks; ++c) n += s_count[c];
   const uint32_t k = static_cast<uint32_t>(p.topk);
   int32_t* dst = p.out_idx + static_cast<size_t>(b) * p.topk;
+  // fn(key, pos, has) for every candidate, in warp-uniform rounds (has = false past a list's end)
   auto for_each = [&](auto&& fn) {
     for (int32_t c = 0; c < p.n_chunks; ++c) {
       const uint32_t* kk = p.part_keys + (base_slot + c) * p.topk;
       const int32_t* pp = p.part_pos + (base_slot + c) * p.topk;
-      for (uint32_t j = tid; j < s_count[c]; j += T) fn(kk[j], pp[j]);
+      for (uint32_t j0 = 0; j0 < s_count[c]; j0 += T) {
+        const uint32_t j = j0 + tid;
+        const bool has = j < s_count[c];
+        fn(has ? kk[j] : 0u, has ? pp[j] : 0, has);
+      }
     }
   };
   uint32_t vk = 0, plim = 0xFFFFFFFFu;
   if (n > k) {
-    uint32_t prefix = 0, mask = 0, rem = k, n_eq = 0;
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    // ---- key passes over an adaptive range: 256 bins over [min, max] of the candidates, then
+    // over the chosen bin, until the bin holding the k-th key is taken whole or is one value
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for_each([&](uint32_t key, int32_t, bool has) {
+      if (has) {
+        lo = min(lo, key);
+        hi = max(hi, key);
+      }
+    });
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) {
+      s_lo[tid >> 5] = lo;
+      s_hi[tid >> 5] = hi;
+    }
+    __syncthreads();
+    for (int w = 0; w < T / 32; ++w) {
+      lo = min(lo, s_lo[w]);
+      hi = max(hi, s_hi[w]);
+    }
+    uint32_t rem = k, shift = bin_shift(hi - lo), a_lo = lo, a_hi = hi;
+    bool ties = false;
+    while (true) {
       for (uint32_t i = tid; i < 256; i += T) sc.hist[i] = 0;
       __syncthreads();
-      for_each([&](uint32_t key, int32_t) {
-        if ((key & mask) == prefix) atomicAdd(&sc.hist[(key >> shift) & 255u], 1u);
+      for_each([&](uint32_t key, int32_t, bool has) {
+        if (has && key >= a_lo && key <= a_hi) atomicAdd(&sc.hist[(key - a_lo) >> shift], 1u);
       });
       __syncthreads();
-      if (tid < 32) scan_pick<true>(&sc, rem);
+      if (tid < 32) scan_bins<true>(&sc, rem);
       __syncthreads();
-      rem -= sc.above;
-      n_eq = sc.hist[sc.bin];
-      prefix |= sc.bin << shift;
-      mask |= 0xFFu << shift;
-      __syncthreads();
+      const uint32_t bin = sc.bin, above = sc.above, cnt = sc.cnt;
+      __syncthreads();                                  // scan results read before the next pass
+      rem -= above;
+      const uint32_t blo = a_lo + (bin << shift);
+      if (cnt == rem) {                                 // the whole bin is in: keys >= blo
+        vk = blo;
+        break;
+      }
+      if (shift == 0) {                                 // one key value, more items than places
+        vk = blo;
+        ties = true;
+        break;
+      }
+      a_hi = bin_end(blo, shift, a_hi);
+      a_lo = blo;
+      shift = shift > 8u ? shift - 8u : 0u;
     }
-    vk = prefix;
-    if (rem < n_eq) {
+    if (ties) {
+      // ---- position passes among the candidates equal to vk: keep the rem lowest positions
       uint32_t pprefix = 0, pmask = 0, prem = rem;
-      for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int ps = 24; ps >= 0; ps -= 8) {
         for (uint32_t i = tid; i < 256; i += T) sc.hist[i] = 0;
         __syncthreads();
-        for_each([&](uint32_t key, int32_t ps) {
-          const uint32_t pu = static_cast<uint32_t>(ps);
-          if (key == vk && (pu & pmask) == pprefix) atomicAdd(&sc.hist[(pu >> shift) & 255u], 1u);
+        for_each([&](uint32_t key, int32_t pos, bool has) {
+          const uint32_t pu = static_cast<uint32_t>(pos);
+          if (has && key == vk && (pu & pmask) == pprefix) atomicAdd(&sc.hist[(pu >> ps) & 255u], 1u);
         });
         __syncthreads();
         if (tid < 32) scan_pick<false>(&sc, prem);
         __syncthreads();
         prem -= sc.above;
-        pprefix |= sc.bin << shift;
-        pmask |= 0xFFu << shift;
+        pprefix |= sc.bin << ps;
+        pmask |= 0xFFu << ps;
         __syncthreads();
       }
       plim = pprefix;
+    } else {
+      plim = 0xFFFFFFFFu;                               // every candidate equal to vk is kept
     }
   }
+  // ---- write the kept positions, one atomic per warp and round
   if (tid == 0) sc.out_count = 0;
   __syncthreads();
   const bool all = n <= k;
-  for_each([&](uint32_t key, int32_t ps) {
-    if (all || key > vk || (key == vk && static_cast<uint32_t>(ps) <= plim)) {
-      const uint32_t at = atomicAdd(&sc.out_count, 1u);
-      if (at < k) dst[at] = ps;
-    }
+  for_each([&](uint32_t key, int32_t ps, bool has) {
+    const bool keep = has && (all || key > vk || (key == vk && static_cast<uint32_t>(ps) <= plim));
+    const uint32_t m = __ballot_sync(0xffffffffu, keep);
+    uint32_t base = 0;
+    if (lane == 0 && m) base = atomicAdd(&sc.out_count, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const uint32_t at = base + __popc(m & ((1u << lane) - 1u));
+    if (keep && at < k) dst[at] = ps;
   });
   __syncthreads();
   for (uint32_t j = min(sc.out_count, k) + tid; j < k; j += T) dst[j] = -1;
