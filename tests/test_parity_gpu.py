@@ -150,6 +150,23 @@ def test_equal_scores_select_the_lowest_positions():
         assert (idx_h[i, n:] == -1).all()
 
 
+def test_decode_equal_scores_merge_by_position():
+    # every index score is 0, so each sequence keeps its lowest min(k, len) positions; with
+    # lengths spanning one to three 8192-key chunks, the merge must resolve the ties across
+    # chunk lists by position, and a sequence shorter than k keeps every key
+    cfg = synthetic.config("decode", batch=4, max_len=20000, len_range=(100, 20000))
+    g = _inputs(cfg, 12)
+    g["w"].zero_()
+    lens = [100, 2048, 9000, 20000]
+    g["lengths"] = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    idx, out, lse = _run_forward(cfg, g)
+    idx_h = idx.cpu().numpy()
+    for b, n_b in enumerate(lens):
+        n = min(cfg.topk, n_b)
+        assert sorted(idx_h[b, 0, :n].tolist()) == list(range(n))
+        assert (idx_h[b, 0, n:] == -1).all()
+
+
 @pytest.mark.parametrize("topk", [1, 7, 2048])
 def test_topk_extremes(topk):
     cfg = synthetic.config("tiny", n_q=260, max_len=260, topk=topk)
