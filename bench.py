@@ -331,8 +331,11 @@ def run_ours(args, cfg, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world)
-    # kernels per step: the indexer is one launch (decode: chunk kernel + merge), the attention one
-    launches = (2 if cfg.is_decode else 1) * int(do_idx) + int(do_att)
+    # kernels per step: the indexer is one launch (decode: chunk kernel + merge), the attention one;
+    # dims other than the production ones add the copies into padded layouts (3 before the
+    # indexer; 2 before and 2 after the attention)
+    padded = (cfg.n_idx_heads, cfg.idx_dim, cfg.n_heads, cfg.d_latent, cfg.d_rope) != (64, 128, 128, 512, 64)
+    launches = ((2 if cfg.is_decode else 1) + (3 if padded else 0)) * int(do_idx) + (1 + (4 if padded else 0)) * int(do_att)
     return dict(total_ms=total_ms, idx_ms=idx_ms, att_ms=att_ms, clocks=clocks, e2e=e2e, launches_per_step=launches)
 
 
@@ -569,7 +572,7 @@ def main():
     ap.add_argument("--steps", type=int, default=None,
                     help="timed steps (default 10; decode: 1000, so clocks are sampled during the timed region)")
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="prefill_128k", choices=["prefill_4k", "prefill_32k", "prefill_128k", "decode"])
+    ap.add_argument("--workload", default="prefill_128k", choices=["tiny", "prefill_4k", "prefill_32k", "prefill_128k", "decode"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=2)
