@@ -7,7 +7,7 @@
 // out of the dot product: both are positive, so this equals sum_j w * ReLU(q . k) on the
 // decoded values), and keeps the k largest per query (Step 2), ties to the lower s.
 //
-// Design (one CTA per SM, persistent over work items):
+// Design (one CTA per SM in prefill, two in decode; persistent over work items):
 //  * a work item is NQ consecutive queries of one sequence and a contiguous key range;
 //  * TMA brings the item's query block [NQ*64 rows x 128 B] once and streams key tiles
 //    [128 keys x 128 B] through a ring of shared-memory stages (128-byte swizzle);
@@ -16,10 +16,11 @@
 //    accumulators, so the MMA of tile i+1 overlaps the epilogue of tile i;
 //  * epilogue warps own one TMEM lane quarter each (a key per thread); they read the
 //    64 head columns of a query, apply ReLU and the weighted head sum in fp32 registers,
-//    mask s > pos(t), and append survivors of the per-query threshold into a candidate
-//    buffer in shared memory. When a buffer nears capacity, all epilogue warps run an exact
-//    radix select that keeps exactly k and raises the threshold. The L x L score matrix is
-//    never written anywhere.
+//    mask s > pos(t), and note which keys beat the query's threshold; every few tiles each
+//    warp appends its survivors to the query's candidate buffer in shared memory with one
+//    atomic. When a buffer nears capacity, the query's warps shrink it (a histogram pass over
+//    the candidates' key range) or select exactly k, which raises the threshold. The L x L
+//    score matrix is never written anywhere.
 //  * prefill items cover a query block's whole causal key range and write the final
 //    indices; decode items (one query per sequence) cover a key chunk and write an exact
 //    partial top-k to the workspace, merged by `merge_partials_kernel`.
