@@ -245,6 +245,13 @@ def rank_seed(seed: int, rank: int) -> int:
     return seed + rank
 
 
+def _free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
 def max_over_ranks(x: float, device) -> float:
     """Max of a per-rank scalar over the process group (the job's time is its slowest rank)."""
     if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
@@ -339,6 +346,97 @@ def run_ours(args, cfg, rank, world, local_rank):
     return dict(total_ms=total_ms, idx_ms=idx_ms, att_ms=att_ms, clocks=clocks, e2e=e2e, launches_per_step=launches)
 
 
+
+
+def _work_rows(cfg, r0, r1):
+    """Algorithmic work of query rows [r0, r1) of one causal prefill sequence."""
+    k = cfg.topk
+
+    def sel(t):                                                  # sum over u < t of min(k, u + 1)
+        return t * (t + 1) // 2 if t <= k else k * (k + 1) // 2 + (t - k) * k
+    pairs = r1 * (r1 + 1) // 2 - r0 * (r0 + 1) // 2
+    sel_rows = sel(r1) - sel(r0)
+    return {"indexer_flop": pairs * 2 * cfg.n_idx_heads * cfg.idx_dim,
+            "attn_flop": sel_rows * 2 * cfg.n_heads * (cfg.d_qk + cfg.d_v),
+            "attn_gather_bytes": sel_rows * cfg.d_qk * 2, "pairs": pairs, "sel_rows": sel_rows}
+
+
+def run_sharded(args, cfg, rank, world, local_rank):
+    """One sequence's query rows split over the ranks (strong scaling).
+
+    Every rank draws the same sequence. It generates only its own rows' query-side inputs and
+    its own tokens' key-side cache rows. The timed step is the all-gather of the key side, then
+    the rank's indexer and attention calls on its rows as one chunk (n_q = r1 - r0, lengths =
+    r1)."""
+    import sparse_attention_long_indexer_b200 as dsa
+    from sparse_attention_long_indexer_b200 import shard
+    import dataclasses
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    seed = args.seed
+    L = cfg.max_len
+    parts = shard.row_partition(L, world, cfg.topk)
+    c = shard.chunk_call(parts, rank)
+    r0, r1 = parts[rank]
+    rows = range(r0, r1)
+    step_q = 8192
+    qc, qs = [], []
+    for a in range(r0, r1, step_q):                      # the query codes in bounded pieces
+        x, y = synthetic.gen_q_idx(cfg, seed, dev, tokens=range(a, min(r1, a + step_q)))
+        qc.append(x)
+        qs.append(y)
+    q_idx = torch.cat(qc) if qc else torch.empty((0, cfg.n_idx_heads, cfg.idx_dim), dtype=torch.uint8, device=dev)
+    q_scale = torch.cat(qs) if qs else torch.empty((0,), dtype=torch.float32, device=dev)
+    w = synthetic.gen_w(cfg, seed, dev, tokens=rows)
+    q = synthetic.gen_q(cfg, seed, dev, tokens=rows)
+    k_loc, ks_loc = synthetic.gen_k_idx(cfg, seed, dev, b=0, s_range=rows)
+    kv_loc = synthetic.gen_kv(cfg, seed, dev, b=0, positions=rows)
+    ccfg = dataclasses.replace(cfg, n_q=c.n_q)
+    dims = dsa.dims_for(ccfg)
+    ws = dsa.Workspace.create(dims, cfg.topk, device=dev)
+    lengths = torch.tensor([c.length], dtype=torch.int32, device=dev)
+    idx = torch.empty((1, c.n_q, cfg.topk), dtype=torch.int32, device=dev)
+    out = torch.empty((1, c.n_q, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((1, c.n_q, cfg.n_heads), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        k_full = shard.all_gather_rows(k_loc, parts).view(1, L, cfg.idx_dim)
+        ks_full = shard.all_gather_rows(ks_loc, parts)
+        kv_full = shard.all_gather_rows(kv_loc, parts).view(1, L, cfg.d_qk)
+        scales = torch.cat([q_scale, ks_full])
+        if ev is not None:
+            ev[1].record(stream)
+        dsa.dsa_indexer_topk(dims, q_idx, w, k_full, scales, lengths, cfg.topk, idx, ws.buf, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        dsa.dsa_sparse_mla_attn(dims, q, kv_full, idx, cfg.topk, out, lse, ws.buf, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ws.check()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    end.record(stream)
+    torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    ws.check()
+    total_ms = max_over_ranks(start.elapsed_time(end), dev)
+    return dict(total_ms=total_ms, gather_ms=[e[0].elapsed_time(e[1]) for e in evs],
+                idx_ms=[e[1].elapsed_time(e[2]) for e in evs], att_ms=[e[2].elapsed_time(e[3]) for e in evs],
+                clocks=clocks, e2e=None, launches_per_step=2, shard={"parts": parts, "rank0_rows": parts[0]})
 
 
 def run_e2e_whole(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
@@ -584,6 +682,9 @@ def main():
     ap.add_argument("--stage", default="all", choices=["all", "indexer", "attention"],
                     help="time one stage only (profiling); the line then reports that stage")
     ap.add_argument("--seq-len", type=int, default=0, help="override L of a prefill workload (profiling)")
+    ap.add_argument("--shard", default="sequences", choices=["sequences", "rows"],
+                    help="N>1: one sequence per rank (weak scaling), or one sequence's query rows split over "
+                         "the ranks with an all-gather of the key-side caches per step (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -606,15 +707,21 @@ def main():
             return 0
         return run_reference(args, cfg, world)
 
-    if world > 1:
+    sharded = args.shard == "rows" and not cfg.is_decode
+    if world > 1 or sharded:
         import datetime
+        if world == 1:                                   # a one-rank group runs the same sharded code
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", str(_free_port()))
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=torch.device("cuda", local_rank))
-    res = run_ours(args, cfg, rank, world, local_rank)
+    res = run_sharded(args, cfg, rank, world, local_rank) if sharded else run_ours(args, cfg, rank, world, local_rank)
     if rank == 0:
         print(json.dumps(report(args, cfg, res, world)), flush=True)
-    if world > 1:
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     return 0
@@ -622,7 +729,9 @@ def main():
 
 def report(args, cfg, res, world):
     peaks = _peaks()
-    w = _work(cfg, rank_seed(args.seed, 0))
+    sh = res.get("shard")
+    # row sharding: rank 0's rows set the per-stage work (the job's time is the slowest rank's)
+    w = _work_rows(cfg, *sh["rank0_rows"]) if sh else _work(cfg, rank_seed(args.seed, 0))
     metric, unit = _metric(cfg)
     ms_step = res["total_ms"] / args.steps
     idx_ms = statistics.mean(res["idx_ms"])
@@ -678,11 +787,23 @@ def report(args, cfg, res, world):
                 "global_batch": cfg.batch * world, "seq_len": cfg.max_len, "topk": cfg.topk,
                 "parallelism": f"{world} independent sequences, one per GPU (no data-path collective)",
                 "l2": "inputs larger than L2 (q alone is %.1f GB)" % (cfg.n_q * cfg.n_heads * cfg.d_qk * 2 / 1e9)}
+    if sh:
+        value = cfg.batch * cfg.n_q * args.steps / (res["total_ms"] / 1e3)      # one sequence per step
+        sizes = [r1 - r0 for r0, r1 in sh["parts"]]
+        conf["global_batch"] = cfg.batch
+        conf["parallelism"] = (f"query rows of one sequence over {world} GPUs (rows per rank {sizes}, balanced by "
+                               f"causal work); one all-gather of the key-side caches per step")
+        key_bytes = cfg.max_len * (cfg.idx_dim + 4 + cfg.d_qk * 2)
+        stages["allgather"] = {"ms": statistics.mean(res["gather_ms"]), "bytes": key_bytes,
+                               "note": "rank 0's view; every rank receives the whole key side"}
+    else:
+        value = aggregate_value(cfg.batch * cfg.n_q, args.steps, world, res["total_ms"])
     line = {
-        "metric": metric, "value": aggregate_value(cfg.batch * cfg.n_q, args.steps, world, res["total_ms"]),
+        "metric": metric, "value": value,
         "unit": unit,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3+bf16 (fp32 accumulate)",
+        "higher_is_better": True, "scaling": "strong" if sh else "weak", "vs_baseline": None,
+        "dtype": "fp8e4m3+bf16 (fp32 accumulate)",
         "data": "synthetic", "config": conf,
         "roofline": roofline, "stages": stages,
         "gpu_launches": res.get("launches_per_step", len(stages)) * args.steps,
