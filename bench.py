@@ -38,6 +38,11 @@ DECODE_METRIC = "DSA decode sequences/s (indexer+top-k+sparse MLA), 64 sequences
 DECODE_UNIT = "sequences/s"
 
 
+def _workload_name(cfg):
+    d = cfg.description
+    return d if d.startswith(cfg.name + ":") else f"{cfg.name}: {d}"
+
+
 def _metric(cfg):
     return (DECODE_METRIC, DECODE_UNIT) if cfg.is_decode else (METRIC, UNIT)
 
@@ -850,7 +855,7 @@ def run_reference(args, cfg, world):
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": f"{cfg.name}: {cfg.description}", "global_batch": cfg.batch,
+            "config": {"workload": _workload_name(cfg), "global_batch": cfg.batch,
                        "seq_len": cfg.max_len, "topk": cfg.topk, "parallelism": "CPU oracle, rank 0 only"},
             "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
