@@ -64,6 +64,7 @@ namespace {
 constexpr uint64_t kWaitBudgetNs = 2000000000ull;   // 2 s per bounded wait
 constexpr size_t kAlign = 256;
 constexpr int kPrefillNQ = 4;                       // queries per prefill indexer work item
+constexpr int kMergeThreads = 1024;                  // decode merge: one CTA per sequence
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -261,7 +262,7 @@ dsa_status run_indexer(const dsa_dims& d, const uint8_t* q_idx, const __nv_bfloa
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return DSA_ERR_CUDA;
     MergeParams mp{p.part_keys, p.part_pos, p.part_count, out_idx, L.n_chunks, topk};
-    merge_partials_kernel<512><<<d.batch, 512, 0, st>>>(mp);
+    merge_partials_kernel<kMergeThreads><<<d.batch, kMergeThreads, 0, st>>>(mp);
     return from_cuda(cudaGetLastError());
   }
   p.n_chunks = 0;
@@ -560,6 +561,6 @@ extern "C" dsa_status dsa_indexer_topk_decode_noalloc(const dsa_dims* dims, cons
   indexer_topk_kernel<1><<<grid, IdxCfg<1>::THREADS, IdxCfg<1>::SMEM_BYTES, st>>>(map_q, map_k, p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   MergeParams mp{p.part_keys, p.part_pos, p.part_count, out_idx, n_chunks, topk};
-  merge_partials_kernel<512><<<d.batch, 512, 0, st>>>(mp);
+  merge_partials_kernel<kMergeThreads><<<d.batch, kMergeThreads, 0, st>>>(mp);
   return from_cuda(cudaGetLastError());
 }
