@@ -58,3 +58,27 @@ def test_prefill_line_keeps_the_headline_metric():
     assert line["metric"] == bench.METRIC and line["unit"] == "query-tokens/s"
     assert line["stages"]["indexer_topk"]["bound"] == "tensor"
     assert line["gpu_launches"] == 20
+
+
+def test_rank_row_work_sums_to_the_sequence():
+    from sparse_attention_long_indexer_b200 import shard
+    cfg = synthetic.config("prefill_32k")
+    parts = shard.row_partition(cfg.n_q, 3, cfg.topk)
+    whole = bench._work(cfg, 0)
+    per = [bench._work_rows(cfg, r0, r1) for r0, r1 in parts]
+    for key in ("pairs", "sel_rows", "indexer_flop", "attn_flop"):
+        assert sum(w[key] for w in per) == whole[key]
+
+
+def test_row_sharded_line_is_strong_scaling_over_the_whole_sequence():
+    from sparse_attention_long_indexer_b200 import shard
+    cfg = synthetic.config("prefill_128k")
+    parts = shard.row_partition(cfg.n_q, 4, cfg.topk)
+    res = dict(_res(2), gather_ms=[0.4] * 10, shard={"parts": parts, "rank0_rows": parts[0]})
+    line = bench.report(_args(), cfg, res, 4)
+    assert line["scaling"] == "strong" and line["n_gpus"] == 4
+    # one sequence per step over the slowest rank's time, not four
+    assert line["value"] == pytest.approx(cfg.n_q * 10 / 0.020)
+    assert line["stages"]["allgather"]["bytes"] == cfg.max_len * (128 + 4 + 576 * 2)
+    w0 = bench._work_rows(cfg, *parts[0])
+    assert line["stages"]["indexer_topk"]["achieved"] == pytest.approx(w0["indexer_flop"] / 1.2e-3 / 1e12)
