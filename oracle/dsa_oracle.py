@@ -26,7 +26,9 @@ Pins (tests/test_oracle_pins.py, CPU only) tie each function to something other
 than itself: the E4M3 and bf16 decoders to torch's own casts on all codes; the
 index score to the identity I(q) - I(-q) = (sum_j w_j q_j) . k (ReLU(x) - ReLU(-x)
 = x), to nonnegativity for w >= 0 and to the one-head / unit-weight special
-case; the selection to a brute-force sort on tiny rows and to causality; the
+case; the per-query driver's application of the per-token FP8 scales to a
+brute-force loop over torch-decoded codes with non-uniform, non-power-of-two key
+scales and a query scale other than one; the selection to a brute-force sort on tiny rows and to causality; the
 attention to torch's scaled_dot_product_attention in float64 when every
 preceding token is selected (k >= pos+1), to weights summing to one, to the
 one-row and equal-logit closed forms and to scipy's logsumexp. Absolute values

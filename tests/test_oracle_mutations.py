@@ -72,7 +72,36 @@ def _e4m3_bias_8(codes, scale=None):
     return od.__dict__["_orig_e4m3"](codes, scale) * 0.5
 
 
+def _driver(q_of, k_of):
+    """indexer_topk_row with the decoding of q and k replaced (planted scale mistakes)."""
+    def row(q_codes, q_scale, w_bits, k_codes, k_scale, pos, topk):
+        if pos < 0:
+            return np.zeros(0, dtype=np.int64), np.zeros(0)
+        q = q_of(q_codes, q_scale)
+        k = k_of(k_codes, np.asarray(k_scale, dtype=np.float64), q_scale, pos)
+        scores = od.index_scores(q, od.decode_bf16(w_bits), k)
+        return od.select_topk(scores, topk).astype(np.int64), scores
+    return row
+
+
+def _q_scaled(q_codes, q_scale):
+    return od.decode_e4m3(q_codes, np.full(q_codes.shape[0], q_scale))
+
+
+MUTANTS_DRIVER = {
+    # keys decoded without their scales
+    "driver_k_scale_dropped": _driver(_q_scaled, lambda kc, ks, qs, pos: od.decode_e4m3(kc[: pos + 1])),
+    # every key takes the scale of the next token
+    "driver_k_scale_shifted": _driver(
+        _q_scaled, lambda kc, ks, qs, pos: od.decode_e4m3(kc[: pos + 1], np.roll(ks, -1)[: pos + 1])),
+    # the query's scale applied to the keys (query unscaled, key scales unused)
+    "driver_q_scale_on_keys": _driver(
+        lambda qc, qs: od.decode_e4m3(qc),
+        lambda kc, ks, qs, pos: od.decode_e4m3(kc[: pos + 1], np.full(pos + 1, qs))),
+}
+
 MUTANTS = {
+    **{n: ("indexer_topk_row", f) for n, f in MUTANTS_DRIVER.items()},
     "relu_after_sum": ("index_scores", _relu_after_sum),
     "no_relu": ("index_scores", _no_relu),
     "unweighted_heads": ("index_scores", _unweighted),
@@ -98,7 +127,7 @@ def _run_pins():
             if params:
                 names = [s.strip() for s in params[0].args[0].split(",")]
                 for vals in params[0].args[1]:
-                    fn(**dict(zip(names, vals)))
+                    fn(**dict(zip(names, vals if len(names) > 1 else (vals,))))
             else:
                 fn()
         except Exception:

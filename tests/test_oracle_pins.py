@@ -121,6 +121,44 @@ def _tiny_row_inputs(cfg, seed, pos):
             k_codes.numpy(), k_scale.numpy())
 
 
+def _finite_e4m3_codes(r, shape):
+    c = r.integers(0, 256, size=shape).astype(np.uint8)
+    c[(c & 0x7F) == 0x7F] ^= 0x01                    # S.1111.111 is NaN: use the neighbouring code
+    return c
+
+
+@pytest.mark.parametrize("pos", [11, 8, 0])
+def test_indexer_row_applies_each_tokens_scale(pos):
+    # One query against 12 keys, each key with its own scale (neither uniform nor a power of two)
+    # and a query scale != 1: the real value of a code is code x its token's scale. Decoded here
+    # with torch's own float8_e4m3fn / bfloat16 casts and summed with explicit loops:
+    #     I[s] = sum_j w_j * max(0, sum_d (q_code[j,d] * s_q) * (k_code[s,d] * s_k[s]))
+    H, d, n, topk = 3, 5, 12, 4
+    r = np.random.default_rng(77 + pos)
+    q_codes, k_codes = _finite_e4m3_codes(r, (H, d)), _finite_e4m3_codes(r, (n, d))
+    q_scale = 0.3716
+    k_scale = r.uniform(0.05, 3.0, size=n)
+    w_bits = torch.tensor(r.standard_normal(H), dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy()
+    w_bits = w_bits.view(np.uint16)
+    tq = torch.from_numpy(q_codes).view(torch.float8_e4m3fn).double().tolist()
+    tk = torch.from_numpy(k_codes).view(torch.float8_e4m3fn).double().tolist()
+    tw = torch.from_numpy(w_bits.view(np.int16)).view(torch.bfloat16).double().tolist()
+    expect = []
+    for s in range(pos + 1):
+        acc = 0.0
+        for j in range(H):
+            dot = 0.0
+            for e in range(d):
+                dot += (tq[j][e] * q_scale) * (tk[s][e] * float(k_scale[s]))
+            acc += tw[j] * max(0.0, dot)
+        expect.append(acc)
+    idx, scores = oracle.indexer_topk_row(q_codes, q_scale, w_bits, k_codes, k_scale, pos, topk)
+    assert scores.shape == (pos + 1,)
+    np.testing.assert_allclose(scores, expect, rtol=1e-12, atol=1e-300)
+    brute = [s for _, s in sorted((-expect[s], s) for s in range(pos + 1))][: min(topk, pos + 1)]
+    assert idx.tolist() == brute
+
+
 def test_selection_is_causal_and_counts_min_k_pos():
     cfg = synthetic.config("tiny")
     for pos in [0, 1, 5, 63, 64, 65, 200, 511]:
