@@ -131,7 +131,9 @@ dsa_status dsa_forward(const dsa_dims* dims, const void* q_idx, const void* w, c
  * array of the library (16 MiB + 4 KiB, held by every GPU that loads the library until the
  * process exits), so the call allocates nothing and needs no workspace.
  *   status  optional device pointer to 2 uint32 words: a device-side error (see dsa_status)
- *           is recorded there, first error wins; the caller zeroes and reads it. May be NULL.
+ *           is recorded there, first error wins; the caller zeroes and reads it. May be NULL,
+ *           but then a device-side error goes unreported: after a bounded wait that ran out,
+ *           the selection of the sequences that were not finished is incomplete without notice.
  * Limits: batch * ceil(max_len / 8192) <= 1024 and topk <= 2048, else DSA_ERR_UNSUPPORTED
  * (also for n_q != 1 or other dims). The first call on a device looks up the array's device
  * address; make that first call before any stream capture. All calls on one device share

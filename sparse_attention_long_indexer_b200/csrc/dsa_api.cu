@@ -547,8 +547,10 @@ extern "C" dsa_status dsa_indexer_topk_decode_noalloc(const dsa_dims* dims, cons
   p.topk = topk;
   p.wait_budget_ns = kWaitBudgetNs;
   p.n_chunks = n_chunks;
-  // the slots are laid out with the call's top-k as row width; every slot a call reads is
-  // written earlier in the same call, so stale contents from a previous call are never used
+  // the slots are laid out with the call's top-k as row width. The chunk kernel zeroes the
+  // count of every slot of this call before it starts, and the merge reads only a slot's first
+  // count entries, so an earlier call's contents are never used: a slot an aborted CTA never
+  // reached counts as empty (the abort itself is reported through `status`)
   p.part_keys = reinterpret_cast<uint32_t*>(scratch);
   p.part_pos = reinterpret_cast<int32_t*>(scratch + kStaticKeysBytes);
   p.part_count = reinterpret_cast<int32_t*>(scratch + 2 * kStaticKeysBytes);

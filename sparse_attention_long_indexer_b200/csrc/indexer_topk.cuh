@@ -194,13 +194,24 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
+  const int32_t G = gridDim.x;
+  const int32_t cta = blockIdx.x;
+  if (NQ == 1) {
+    // decode: slot u of the partial lists belongs to work item u, which only this CTA runs.
+    // Its count starts at zero here, before the barrier, so a slot this CTA never reaches
+    // (after an aborted wait) reads as empty in the merge instead of holding an earlier
+    // call's count.
+    for (int32_t r = static_cast<int32_t>(threadIdx.x);; r += static_cast<int32_t>(blockDim.x)) {
+      const int32_t u = item_of(r, cta, G);
+      if (u >= p.n_items) break;
+      p.part_count[u] = 0;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   Waiter wt{p.status, abort_flag, p.wait_budget_ns, 1u};
-  const int32_t G = gridDim.x;
-  const int32_t cta = blockIdx.x;
 
   if (warp == C::PRODUCER_WARP) {
     // ------------------------------------------------------------- TMA producer
@@ -528,7 +539,9 @@ __global__ void __launch_bounds__(T) merge_partials_kernel(const MergeParams p) 
   const uint32_t tid = threadIdx.x, lane = tid & 31u;
   const int32_t b = blockIdx.x;
   const size_t base_slot = static_cast<size_t>(b) * p.n_chunks;
-  for (int32_t c = tid; c < p.n_chunks; c += T) s_count[c] = static_cast<uint32_t>(p.part_count[base_slot + c]);
+  // a count never exceeds topk; the clamp keeps every read inside its slot regardless
+  for (int32_t c = tid; c < p.n_chunks; c += T)
+    s_count[c] = min(static_cast<uint32_t>(max(p.part_count[base_slot + c], 0)), static_cast<uint32_t>(p.topk));
   __syncthreads();
   uint32_t n = 0;
   for (int32_t c = 0; c < p.n_chunks; ++c) n += s_count[c];

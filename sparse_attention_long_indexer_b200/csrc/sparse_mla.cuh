@@ -612,13 +612,16 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
           l *= alpha;
         }
         // P = 2^(s*sc - m2) in bf16 for the output product; the row sum adds the same bf16 values,
-        // so the normalisation matches the weights the output product uses
+        // so the normalisation matches the weights the output product uses. While every row seen so
+        // far was masked, m2 is still -inf and so is every logit of this block: the subtrahend is
+        // then 0, so P = 2^-inf = 0 instead of the NaN of -inf + inf.
+        const float msub = (m2 == -INFINITY) ? 0.0f : m2;
         uint32_t pk[16];
         float2 lsum2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float e0 = ex2_approx(fmaf(__uint_as_float(sr[2 * j]), sc, -m2));
-          const float e1 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 1]), sc, -m2));
+          const float e0 = ex2_approx(fmaf(__uint_as_float(sr[2 * j]), sc, -msub));
+          const float e1 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 1]), sc, -msub));
           const __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
           const float2 back = __bfloat1622float2(pr);
           lsum2.x += back.x;

@@ -39,7 +39,7 @@ import torch
 
 __all__ = [
     "DSAConfig", "CONFIGS", "config", "mix32_int", "normal_rows", "lengths",
-    "quantize_e4m3_rows", "gen_q_idx", "gen_k_idx", "gen_w", "gen_q", "gen_kv",
+    "quantize_e4m3_rows", "quantize_e4m3_rows_amax", "gen_q_idx", "gen_k_idx", "gen_w", "gen_q", "gen_kv",
     "gen_all", "TENSOR_IDS",
 ]
 
@@ -79,6 +79,9 @@ class DSAConfig:
     w_std: float = 0.125
     qkv_std: float = 1.0
     len_range: Optional[tuple] = None   # decode: lengths ~ U[lo, hi] (inclusive)
+    # per-token FP8 scale: "pow2" = the power of two above amax/256 (exact scaling), or
+    # "amax" = amax/448 rounded to fp32 (a general positive scale; generate on the CPU)
+    fp8_scale: str = "pow2"
     description: str = field(default="", compare=False)
 
     @property
@@ -211,6 +214,28 @@ def quantize_e4m3_rows(x: torch.Tensor):
     return y.to(torch.float8_e4m3fn).view(torch.uint8), scale
 
 
+def quantize_e4m3_rows_amax(x: torch.Tensor):
+    """Per-row FP8 E4M3 codes (uint8) and fp32 scales scale = amax / 448.
+
+    The scale is amax/448 computed in float64 and rounded to fp32 (1 if amax == 0), so it is
+    in general not a power of two. Codes are x / scale computed in float64, clamped to
+    [-448, 448], rounded to fp32 and then to E4M3 (round to nearest even). Deterministic on
+    the CPU; tests generate these inputs there and upload them.
+    """
+    amax = x.abs().amax(dim=1).double()
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax)).float()
+    y = (x.double() / scale.double()[:, None]).clamp(-E4M3_MAX, E4M3_MAX).float()
+    return y.to(torch.float8_e4m3fn).view(torch.uint8), scale
+
+
+def _quantizer(cfg: "DSAConfig"):
+    if cfg.fp8_scale == "pow2":
+        return quantize_e4m3_rows
+    if cfg.fp8_scale == "amax":
+        return quantize_e4m3_rows_amax
+    raise ValueError(f"unknown fp8_scale {cfg.fp8_scale!r}")
+
+
 # ----------------------------------------------------------------------------- lengths
 def lengths(cfg: DSAConfig, seed: int) -> torch.Tensor:
     """int32 [B]: L for prefill, U[lo, hi] (seeded) for decode."""
@@ -241,10 +266,10 @@ def gen_q_idx(cfg: DSAConfig, seed: int, device="cpu", tokens=None):
         per = max(1, _CHUNK // rl)
         for a in range(0, n, per):
             b = min(n, a + per)
-            c, s = quantize_e4m3_rows(normal_rows(seed, "q_idx", range(a, b), rl, cfg.q_idx_std, device))
+            c, s = _quantizer(cfg)(normal_rows(seed, "q_idx", range(a, b), rl, cfg.q_idx_std, device))
             codes[a:b], scale[a:b] = c, s
     else:
-        codes, scale = quantize_e4m3_rows(normal_rows(seed, "q_idx", tokens, rl, cfg.q_idx_std, device))
+        codes, scale = _quantizer(cfg)(normal_rows(seed, "q_idx", tokens, rl, cfg.q_idx_std, device))
     return codes.view(-1, cfg.n_idx_heads, cfg.idx_dim), scale
 
 
@@ -261,12 +286,12 @@ def gen_k_idx(cfg: DSAConfig, seed: int, device="cpu", b: Optional[int] = None, 
         per = max(1, _CHUNK // rl)
         for a in range(0, n, per):
             e = min(n, a + per)
-            c, s = quantize_e4m3_rows(normal_rows(seed, "k_idx", range(a, e), rl, cfg.k_idx_std, device))
+            c, s = _quantizer(cfg)(normal_rows(seed, "k_idx", range(a, e), rl, cfg.k_idx_std, device))
             codes[a:e], scale[a:e] = c, s
         return codes.view(cfg.batch, cfg.max_len, rl), scale.view(cfg.batch, cfg.max_len)
     s_range = range(cfg.max_len) if s_range is None else s_range
     rows = range(b * cfg.max_len + s_range.start, b * cfg.max_len + s_range.stop)
-    return quantize_e4m3_rows(normal_rows(seed, "k_idx", rows, rl, cfg.k_idx_std, device))
+    return _quantizer(cfg)(normal_rows(seed, "k_idx", rows, rl, cfg.k_idx_std, device))
 
 
 def _bf16_rows(seed, tensor, rows, row_len, std, device):

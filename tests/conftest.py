@@ -21,3 +21,20 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Near-tie report of the parity tests: per configuration, the query rows checked, the rows
+    whose GPU selection differs from the oracle's exact set (every difference inside the
+    near-tie band), the swapped pairs, and the rows where the band's near-zero floor decided."""
+    try:
+        from tests.dsa_cases import NEAR_TIE_REPORT
+    except Exception:
+        return
+    if not NEAR_TIE_REPORT:
+        return
+    terminalreporter.write_sep("-", "near-tie report (selection parity)")
+    terminalreporter.write_line(f"{'configuration':<28} {'rows':>8} {'rows with swaps':>16} {'pairs':>8} "
+                                f"{'floor used':>11}")
+    for name, (rows, swapped_rows, pairs, floor) in sorted(NEAR_TIE_REPORT.items()):
+        terminalreporter.write_line(f"{name:<28} {rows:>8} {swapped_rows:>16} {pairs:>8} {floor:>11}")

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import synthetic
-from tests.dsa_cases import RowOracle, check_selection, compare_attention
+from tests.dsa_cases import RowOracle, check_selection, compare_attention, report_near_ties
 
 pytestmark = pytest.mark.gpu
 
@@ -32,23 +32,55 @@ def _run_forward(cfg, g, return_idx=True):
     return idx, out, lse
 
 
-def _check_rows(cfg, seed, rows, idx, out, lse, ro=None, attn_rows=None):
+def _rows_to_host(t, rows):
+    """t[b, i] for the listed (b, i), gathered on the device first, as float64/int numpy."""
+    if not rows:
+        return np.zeros((0,) + tuple(t.shape[2:]))
+    bi = torch.tensor([b for b, _ in rows], device=t.device)
+    ii = torch.tensor([i for _, i in rows], device=t.device)
+    sel = t[bi, ii]
+    return sel.cpu().numpy() if sel.dtype == torch.int32 else sel.double().cpu().numpy()
+
+
+def _check_rows(cfg, seed, rows, idx, out, lse, ro=None, attn_rows=None, name=None):
+    """Selections of ``rows`` against the oracle (near-ties allowed), and the attention of
+    ``attn_rows`` (default: all of them) against the oracle's attention over the GPU's own sets.
+    Returns {(b, i): the oracle's exact selection} for reuse."""
     ro = ro or RowOracle(cfg, seed)
-    idx_h = idx.cpu().numpy()
-    out_h = out.float().cpu().numpy()
-    lse_h = lse.cpu().numpy()
-    ties = 0
-    att_gpu, att_ref, lse_gpu, lse_ref = [], [], [], []
-    for (b, i) in rows:
+    idx_h = _rows_to_host(idx, rows)
+    stats, sets = [], {}
+    for r, (b, i) in enumerate(rows):
         sel_o, scores = ro.indexer(b, i)
-        ties += check_selection(idx_h[b, i], scores, cfg.topk, ro.pos(b, i))
-        if attn_rows is None or (b, i) in attn_rows:
-            o, l = ro.attention(b, i, idx_h[b, i])          # oracle attention over the GPU's own set
-            att_gpu.append(out_h[b, i]); att_ref.append(o)
-            lse_gpu.append(lse_h[b, i]); lse_ref.append(l)
-    if att_gpu:
-        compare_attention(np.stack(att_gpu), np.stack(lse_gpu), np.stack(att_ref), np.stack(lse_ref))
-    return ties
+        sets[(b, i)] = sel_o
+        stats.append(check_selection(idx_h[r], scores, cfg.topk, ro.pos(b, i)))
+    report_near_ties(name or cfg.name, len(rows), stats)
+    a_rows = [x for x in rows if attn_rows is None or x in attn_rows]
+    if a_rows:
+        out_h, lse_h = _rows_to_host(out, a_rows), _rows_to_host(lse, a_rows)
+        pos = {x: r for r, x in enumerate(rows)}
+        ref = [ro.attention(b, i, idx_h[pos[(b, i)]]) for (b, i) in a_rows]
+        compare_attention(out_h, lse_h, np.stack([r[0] for r in ref]), np.stack([r[1] for r in ref]))
+    return sets
+
+
+def _attention_on_oracle_sets(cfg, g, sets, ro, out=None, lse=None):
+    """The attention kernel fed the oracle's own selections (the other rows select nothing),
+    compared with the oracle's attention over the same sets, row by row."""
+    idx = torch.full((cfg.batch, cfg.n_q, cfg.topk), -1, dtype=torch.int32)
+    for (b, i), s in sets.items():
+        idx[b, i, :len(s)] = torch.from_numpy(np.asarray(s, dtype=np.int32))
+    dims = dsa.dims_for(cfg)
+    ws = dsa.Workspace.create(dims, cfg.topk)
+    if out is None:
+        out, lse = dsa.sparse_mla_attn(dims, g["q"], g["kv"], idx.cuda(), cfg.topk, ws)
+    else:                                   # reuse the caller's output buffers (128K: 17 GB)
+        dsa.dsa_sparse_mla_attn(dims, g["q"], g["kv"], idx.cuda(), cfg.topk, out, lse, ws.buf)
+    torch.cuda.synchronize()
+    ws.check()
+    rows = sorted(sets)
+    ref = [ro.attention(b, i, sets[(b, i)]) for (b, i) in rows]
+    compare_attention(_rows_to_host(out, rows), _rows_to_host(lse, rows), np.stack([r[0] for r in ref]),
+                      np.stack([r[1] for r in ref]))
 
 
 # ----------------------------------------------------------------------------- tiny (all rows)
@@ -63,18 +95,7 @@ def test_tiny_attention_on_oracle_sets():
     cfg = synthetic.config("tiny")
     g = _inputs(cfg, 2, gen_device="cpu")
     ro = RowOracle(cfg, 2)
-    sets = np.full((1, cfg.n_q, cfg.topk), -1, dtype=np.int32)
-    for i in range(cfg.n_q):
-        s, _ = ro.indexer(0, i)
-        sets[0, i, :len(s)] = s
-    dims = dsa.dims_for(cfg)
-    ws = dsa.Workspace.create(dims, cfg.topk)
-    out, lse = dsa.sparse_mla_attn(dims, g["q"], g["kv"], torch.from_numpy(sets).cuda(), cfg.topk, ws)
-    torch.cuda.synchronize()
-    ws.check()
-    ref = [ro.attention(0, i, sets[0, i]) for i in range(cfg.n_q)]
-    compare_attention(out.float().cpu().numpy()[0], lse.cpu().numpy()[0], np.stack([r[0] for r in ref]),
-                      np.stack([r[1] for r in ref]))
+    _attention_on_oracle_sets(cfg, g, {(0, i): ro.indexer(0, i)[0] for i in range(cfg.n_q)}, ro)
 
 
 # ----------------------------------------------------------------------------- 4K (all rows)
@@ -92,38 +113,34 @@ def test_prefill_4k_attention_on_oracle_sets():
     g = _inputs(cfg, 4)
     ro = RowOracle(cfg, 4)
     rows = synthetic.sample_rows(cfg.n_q, 96, 4, extra=[0, 1, 2047, 2048, cfg.n_q - 1])
-    sets = np.full((1, cfg.n_q, cfg.topk), -1, dtype=np.int32)
-    for i in rows:
-        s, _ = ro.indexer(0, i)
-        sets[0, i, :len(s)] = s
-    dims = dsa.dims_for(cfg)
-    ws = dsa.Workspace.create(dims, cfg.topk)
-    out, lse = dsa.sparse_mla_attn(dims, g["q"], g["kv"], torch.from_numpy(sets).cuda(), cfg.topk, ws)
-    torch.cuda.synchronize()
-    ws.check()
-    ref = [ro.attention(0, i, sets[0, i]) for i in rows]
-    compare_attention(out.float().cpu().numpy()[0, rows], lse.cpu().numpy()[0, rows],
-                      np.stack([r[0] for r in ref]), np.stack([r[1] for r in ref]))
+    _attention_on_oracle_sets(cfg, g, {(0, i): ro.indexer(0, i)[0] for i in rows}, ro)
 
 
 # ----------------------------------------------------------------------------- 32K / 128K (sampled rows)
 def test_prefill_32k_sampled_rows():
+    """512 seeded rows plus the first and last 64: selections and attention over the GPU's sets,
+    then the attention kernel fed the oracle's sets of the same rows."""
     cfg = synthetic.config("prefill_32k")
     g = _inputs(cfg, 5)
     idx, out, lse = _run_forward(cfg, g)
     rows = synthetic.sample_rows(cfg.n_q, 512, 5, extra=list(range(64)) + list(range(cfg.n_q - 64, cfg.n_q)))
-    attn = set((0, i) for i in rows[::4])
-    _check_rows(cfg, 5, [(0, i) for i in rows], idx, out, lse, attn_rows=attn)
+    ro = RowOracle(cfg, 5)
+    sets = _check_rows(cfg, 5, [(0, i) for i in rows], idx, out, lse, ro=ro)
+    _attention_on_oracle_sets(cfg, g, sets, ro, out=out, lse=lse)
 
 
 def test_prefill_128k_sampled_rows():
+    """256 seeded rows (plus the first and last): selections, attention over the GPU's sets and
+    over the oracle's sets, at the metric's workload."""
     cfg = synthetic.config("prefill_128k")
     g = _inputs(cfg, 6)
     idx, out, lse = _run_forward(cfg, g)
     rows = synthetic.sample_rows(cfg.n_q, 256, 6, extra=[0, cfg.n_q - 1])
-    attn = set((0, i) for i in rows[::4])
-    _check_rows(cfg, 6, [(0, i) for i in rows], idx, out, lse, attn_rows=attn)
-    del g, idx, out, lse
+    ro = RowOracle(cfg, 6)
+    sets = _check_rows(cfg, 6, [(0, i) for i in rows], idx, out, lse, ro=ro)
+    del idx
+    _attention_on_oracle_sets(cfg, g, sets, ro, out=out, lse=lse)
+    del g, out, lse
     torch.cuda.empty_cache()
 
 
@@ -132,7 +149,9 @@ def test_decode_all_sequences():
     cfg = synthetic.config("decode")
     g = _inputs(cfg, 7)
     idx, out, lse = _run_forward(cfg, g)
-    _check_rows(cfg, 7, [(b, 0) for b in range(cfg.batch)], idx, out, lse)
+    ro = RowOracle(cfg, 7)
+    sets = _check_rows(cfg, 7, [(b, 0) for b in range(cfg.batch)], idx, out, lse, ro=ro)
+    _attention_on_oracle_sets(cfg, g, sets, ro, out=out, lse=lse)
     del g
     torch.cuda.empty_cache()
 
@@ -172,7 +191,7 @@ def test_topk_extremes(topk):
     cfg = synthetic.config("tiny", n_q=260, max_len=260, topk=topk)
     g = _inputs(cfg, 9, gen_device="cpu")
     idx, out, lse = _run_forward(cfg, g)
-    _check_rows(cfg, 9, [(0, i) for i in range(cfg.n_q)], idx, out, lse)
+    _check_rows(cfg, 9, [(0, i) for i in range(cfg.n_q)], idx, out, lse, name=f"tiny L=260 k={topk}")
 
 
 def test_ragged_batch_prefill_with_empty_sequence():
@@ -183,7 +202,7 @@ def test_ragged_batch_prefill_with_empty_sequence():
     idx, out, lse = _run_forward(cfg, g)
     ro = RowOracle(cfg, 10, lengths=lengths)
     rows = [(b, i) for b in range(3) for i in range(cfg.n_q)]
-    _check_rows(cfg, 10, rows, idx, out, lse, ro=ro)
+    _check_rows(cfg, 10, rows, idx, out, lse, ro=ro, name="tiny ragged batch of 3")
     # queries before the start of a short sequence select nothing: out = 0, lse = -inf
     assert (idx[2] == -1).all() and (out[2] == 0).all() and torch.isinf(lse[2]).all()
 
@@ -209,6 +228,119 @@ def test_attention_skips_padding_and_reports_out_of_range():
     st, _ = dsa.dsa_get_device_status(ws.buf)
     assert st == dsa.DSA_ERR_INDEX_RANGE
     assert dsa.dsa_get_device_status(ws.buf)[0] == dsa.DSA_OK    # cleared by the read
+
+
+def test_attention_masked_leading_blocks():
+    """Index rows whose first 64-entry blocks hold no attended entry (padding or entries past
+    max_len), an all-padding row, and padding scattered through a row: masked entries are
+    skipped wherever they appear, with no NaN, and an entry past max_len is reported."""
+    cfg = synthetic.config("tiny", n_q=9, max_len=300, topk=256)
+    g = _inputs(cfg, 16, gen_device="cpu")
+    r = np.random.default_rng(16)
+    k, L = cfg.topk, cfg.max_len
+    rows = np.full((cfg.n_q, k), -1, dtype=np.int32)
+
+    def valid(n):
+        return r.integers(0, L, size=n).astype(np.int32)
+
+    rows[0, 64:84] = valid(20)                      # block 0 all padding
+    rows[1, 130:170] = valid(40)                    # blocks 0-1 and half of block 2 padding
+    rows[2, :64] = L + 7                            # block 0 entirely past max_len (reported)
+    rows[2, 64:94] = valid(30)
+    # row 3: all padding -> out = 0, lse = -inf
+    m = r.random(k) < 0.4                           # padding scattered, block 0 all padding
+    m[:64] = False
+    rows[4, m] = valid(int(m.sum()))
+    rows[5, 192:] = valid(64)                       # only the last block attended
+    rows[6, :3] = valid(3)                          # block 0 partly attended (then padding)
+    rows[7] = valid(k)                              # every entry attended
+    rows[8, 63] = valid(1)[0]                       # one attended entry, the last of block 0
+    rows[8, 64:128] = L + 1                         # then a block past max_len
+    dims = dsa.dims_for(cfg)
+    ws = dsa.Workspace.create(dims, cfg.topk)
+    out, lse = dsa.sparse_mla_attn(dims, g["q"], g["kv"], torch.from_numpy(rows).reshape(1, cfg.n_q, k).cuda(),
+                                   cfg.topk, ws)
+    torch.cuda.synchronize()
+    st, _ = dsa.dsa_get_device_status(ws.buf)
+    assert st == dsa.DSA_ERR_INDEX_RANGE
+    ro = RowOracle(cfg, 16)
+    out_h, lse_h = out.double().cpu().numpy()[0], lse.cpu().numpy()[0]
+    assert not np.isnan(out_h).any() and not np.isnan(lse_h).any()
+    for i in range(cfg.n_q):
+        kept = [int(x) for x in rows[i] if 0 <= x < L]
+        o, l = ro.attention(0, i, kept)
+        compare_attention(out_h[i], lse_h[i], o, l)
+    assert (out_h[3] == 0).all() and np.isneginf(lse_h[3]).all()
+
+
+def test_general_fp8_scales_tiny_forward():
+    """FP8 inputs quantised with scale = amax/448 (not a power of two), so the kernel's fp32
+    folding of the query scale into the head weights and its key-scale multiply round."""
+    cfg = synthetic.config("tiny", fp8_scale="amax")
+    g = _inputs(cfg, 13, gen_device="cpu")
+    m, _ = np.frexp(g["k_scale"].double().cpu().numpy())
+    assert (m != 0.5).mean() > 0.9
+    idx, out, lse = _run_forward(cfg, g)
+    _check_rows(cfg, 13, [(0, i) for i in range(cfg.n_q)], idx, out, lse, name="tiny, amax/448 scales")
+
+
+def test_general_fp8_scales_prefill_4k_indexer():
+    cfg = synthetic.config("prefill_4k", fp8_scale="amax")
+    g = {}
+    g["q_idx"], g["q_scale"] = synthetic.gen_q_idx(cfg, 14)
+    g["k_idx"], g["k_scale"] = synthetic.gen_k_idx(cfg, 14)
+    g["w"] = synthetic.gen_w(cfg, 14)
+    g = {n: v.cuda() for n, v in g.items()}
+    dims = dsa.dims_for(cfg)
+    ws = dsa.Workspace.create(dims, cfg.topk)
+    idx = dsa.indexer_topk(dims, g["q_idx"].view(1, cfg.n_q, cfg.n_idx_heads, cfg.idx_dim), g["w"],
+                           g["k_idx"], g["q_scale"], g["k_scale"], synthetic.lengths(cfg, 14).cuda(), cfg.topk, ws)
+    torch.cuda.synchronize()
+    ws.check()
+    rows = synthetic.sample_rows(cfg.n_q, 768, 14, extra=[0, 1, 2046, 2047, 2048, 2049, cfg.n_q - 1])
+    _check_rows(cfg, 14, [(0, i) for i in rows], idx, None, None, attn_rows=set(),
+                name="prefill_4k, amax/448 scales")
+
+
+def test_row_sharded_chunks_match_the_oracle():
+    """The query-row sharding of one sequence over three ranks, run here as the three ranks'
+    chunk calls on one GPU (n_q = r1 - r0, lengths = r1, the whole key side): sampled rows of
+    every part, and each part's first and last row, against the oracle at their positions."""
+    from sparse_attention_long_indexer_b200 import shard
+    cfg = synthetic.config("prefill_4k")
+    seed = 15
+    g = _inputs(cfg, seed)
+    ro = RowOracle(cfg, seed)
+    parts = shard.row_partition(cfg.max_len, 3, cfg.topk)
+    assert all(r1 > r0 for r0, r1 in parts)
+    k_scale = g["k_scale"].reshape(-1)
+    for rank in range(3):
+        c = shard.chunk_call(parts, rank)
+        r0 = c.row0
+        dims_c = dsa.make_dims(1, c.n_q, cfg.max_len, cfg.n_idx_heads, cfg.idx_dim, cfg.n_heads, cfg.d_latent,
+                               cfg.d_rope, cfg.softmax_scale)
+        ws = dsa.Workspace.create(dims_c, cfg.topk)
+        idx = torch.empty((1, c.n_q, cfg.topk), dtype=torch.int32, device="cuda")
+        out = torch.empty((1, c.n_q, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((1, c.n_q, cfg.n_heads), dtype=torch.float32, device="cuda")
+        scales = torch.cat([g["q_scale"].reshape(-1)[r0:r0 + c.n_q], k_scale]).contiguous()
+        dsa.dsa_forward(dims_c, g["q_idx"][:, r0:r0 + c.n_q].contiguous(), g["w"][:, r0:r0 + c.n_q].contiguous(),
+                        g["k_idx"], scales, torch.tensor([c.length], dtype=torch.int32, device="cuda"), cfg.topk,
+                        g["q"][:, r0:r0 + c.n_q].contiguous(), g["kv"], idx, out, lse, ws.buf)
+        torch.cuda.synchronize()
+        ws.check()
+        local = sorted(set(synthetic.sample_rows(c.n_q, 40, seed + rank, extra=[0, c.n_q - 1])))
+        idx_h = _rows_to_host(idx, [(0, i) for i in local])
+        out_h = _rows_to_host(out, [(0, i) for i in local])
+        lse_h = _rows_to_host(lse, [(0, i) for i in local])
+        stats, refs = [], []
+        for j, i in enumerate(local):
+            t = r0 + i                                   # the row's position in the whole sequence
+            _, scores = ro.indexer(0, t)
+            stats.append(check_selection(idx_h[j], scores, cfg.topk, t))
+            refs.append(ro.attention(0, t, idx_h[j]))
+        report_near_ties("prefill_4k, 3 row shards", len(local), stats)
+        compare_attention(out_h, lse_h, np.stack([x[0] for x in refs]), np.stack([x[1] for x in refs]))
 
 
 def test_empty_problem_is_a_no_op():

@@ -63,6 +63,33 @@ def test_e4m3_quantisation_uses_exact_power_of_two_scales():
     assert torch.equal(ref, codes)
 
 
+def test_e4m3_quantisation_with_amax_scales():
+    x = synthetic.normal_rows(4, "k_idx", range(0, 64), 128, 1.0)
+    x[7] = 0.0
+    codes, scale = synthetic.quantize_e4m3_rows_amax(x)
+    s = scale.double().numpy()
+    xd = x.double().numpy()
+    amax = np.abs(xd).max(1)
+    nz = amax > 0
+    assert (s > 0).all() and (s[~nz] == 1).all()
+    np.testing.assert_allclose(s[nz], amax[nz] / 448.0, rtol=2.0 ** -24)   # amax/448 rounded to fp32
+    m, _ = np.frexp(s[nz])
+    assert (m != 0.5).sum() > 50                                            # general, not powers of two
+    dec = oracle.decode_e4m3(codes.numpy(), scale.numpy())
+    assert np.isfinite(dec).all() and (np.abs(dec) <= 448.0 * s[:, None] * (1 + 2.0 ** -20)).all()
+    # within half an E4M3 step (plus the fp32 rounding of x / scale) of the exact value
+    err = np.abs(dec - xd)
+    assert (err <= np.maximum(np.abs(xd) * 2.0 ** -4, s[:, None] * 2.0 ** -10) * (1 + 1e-6) + 1e-30).all()
+    # the row maximum maps to the top code
+    top = np.abs(oracle.decode_e4m3(codes.numpy()))[nz].max(1)
+    assert (top == 448.0).all()
+    cfg = synthetic.config("tiny", n_q=16, max_len=16, fp8_scale="amax")
+    qc, qs = synthetic.gen_q_idx(cfg, 2)
+    ref_c, ref_s = synthetic.quantize_e4m3_rows_amax(
+        synthetic.normal_rows(2, "q_idx", range(0, 16), cfg.n_idx_heads * cfg.idx_dim, cfg.q_idx_std))
+    assert torch.equal(qc.reshape(16, -1), ref_c) and torch.equal(qs, ref_s)
+
+
 def test_row_subsets_match_full_generation():
     cfg = synthetic.config("tiny", n_q=48, max_len=48)
     g = synthetic.gen_all(cfg, 9)

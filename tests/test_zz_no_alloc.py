@@ -4,9 +4,11 @@ Some callers cannot allocate device memory for a call -- serving runtimes that p
 buffer ahead, plugin interfaces that hand a kernel only its inputs and outputs, loops that
 cannot afford cudaMalloc's implicit synchronisation. This entry point keeps its scratch (the
 per-chunk top-k lists of the decode selection) in a device array inside the library. The test
-calls it through the C ABI and checks its selections against the workspace entry point,
-dsa_indexer_topk, on two calls in a row with different inputs, so leftovers of the first call
-in the shared array cannot go unnoticed. It also checks that oversized problems are refused.
+calls it through the C ABI twice in a row and checks each call's selections against the
+workspace entry point, dsa_indexer_topk, and a few sequences of each against the oracle. The
+first call uses top-k 2048 over five 8192-key chunks per sequence, the second top-k 64 over two
+chunks, so the second call's slots sit where the first left longer lists and larger counts:
+leftovers in the shared array would show. It also checks that oversized problems are refused.
 """
 import ctypes
 
@@ -33,12 +35,14 @@ def _p(t):
 
 
 def test_noalloc_decode_matches_workspace_entry_point():
+    from tests.dsa_cases import RowOracle, check_selection
     dsa, lib = _lib()
-    cfg = synthetic.config("decode", batch=6, max_len=40000, len_range=(3000, 40000))
-    dims = dsa.dims_for(cfg)
-    ws = dsa.Workspace.create(dims, cfg.topk)
     stream = torch.cuda.current_stream()
-    for seed in (31, 32):                               # two calls in a row, different inputs
+    calls = [(31, synthetic.config("decode", batch=6, max_len=40000, len_range=(3000, 40000))),
+             (32, synthetic.config("decode", batch=6, max_len=9000, len_range=(1000, 9000), topk=64))]
+    for seed, cfg in calls:                              # two calls in a row, different inputs and sizes
+        dims = dsa.dims_for(cfg)
+        ws = dsa.Workspace.create(dims, cfg.topk)
         g = synthetic.gen_all(cfg, seed, "cuda")
         scales = torch.cat([g["q_scale"].reshape(-1), g["k_scale"].reshape(-1)]).contiguous()
         ref = dsa.indexer_topk(dims, g["q_idx"], g["w"], g["k_idx"], g["q_scale"], g["k_scale"], g["lengths"],
@@ -53,11 +57,16 @@ def test_noalloc_decode_matches_workspace_entry_point():
         ws.check()
         assert status.tolist() == [0, 0]
         lengths = g["lengths"].tolist()
+        got_all = out.cpu().numpy()
         for b in range(cfg.batch):
             n = min(cfg.topk, lengths[b])
-            got, exp = out[b, 0].tolist(), ref[b, 0].tolist()
+            got, exp = got_all[b, 0].tolist(), ref[b, 0].tolist()
             assert sorted(got[:n]) == sorted(exp[:n])          # same selected set
             assert all(x == -1 for x in got[n:])               # padding after the selection
+        ro = RowOracle(cfg, seed)
+        for b in (0, cfg.batch - 1):                           # and the oracle agrees, up to near-ties
+            _, scores = ro.indexer(b, 0)
+            check_selection(got_all[b, 0], scores, cfg.topk, ro.pos(b, 0))
 
 
 def test_noalloc_decode_refuses_sizes_beyond_its_array():
