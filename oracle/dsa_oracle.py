@@ -31,7 +31,11 @@ brute-force loop over torch-decoded codes with non-uniform, non-power-of-two key
 scales and a query scale other than one; the selection to a brute-force sort on tiny rows and to causality; the
 attention to torch's scaled_dot_product_attention in float64 when every
 preceding token is selected (k >= pos+1), to weights summing to one, to the
-one-row and equal-logit closed forms and to scipy's logsumexp. Absolute values
+one-row and equal-logit closed forms and to scipy's logsumexp; the
+indexer-alignment loss to explicit loops (per-head softmax, head sum, L1
+normalisation, KL), to scipy's softmax and relative entropy, to its closed forms
+(zero for scores = ln p + c, two points, one-hot) and to Gibbs' inequality, and
+its per-query term to padding and order invariance. Absolute values
 at the production shapes have no printed example on the pages: beyond these
 invariants and reductions they are parity-unpinned by the pages.
 """
@@ -42,6 +46,7 @@ import numpy as np
 __all__ = [
     "decode_e4m3", "decode_bf16", "index_scores", "select_topk", "sparse_mla_attention",
     "indexer_topk_row", "sparse_mla_attn_row", "dsa_row",
+    "attention_head_sum_target", "indexer_kl", "indexer_kl_row",
 ]
 
 
@@ -179,3 +184,60 @@ def dsa_row(q_codes, q_scale, w_bits, k_codes, k_scale, q_bits, kv_bits, pos, to
     idx, scores = indexer_topk_row(q_codes, q_scale, w_bits, k_codes, k_scale, pos, topk)
     out, lse = sparse_mla_attn_row(q_bits, kv_bits, idx, d_v, tau)
     return idx, out, lse, scores
+
+
+# ----------------------------------------------------------------------------- indexer alignment loss
+def attention_head_sum_target(q_t: np.ndarray, kv_rows: np.ndarray, tau: float) -> np.ndarray:
+    """Target distribution of the indexer-alignment loss for one query token.
+
+    a[s] = sum_h softmax_s(tau * q[h] . kv[s]) over the rows given, then p = a / sum_s a[s].
+
+    [blog] section "訓練", Step 1 (dense warm-up): for the t-th query token the main
+    attention scores are summed over all heads and the sum is L1-normalised along the
+    sequence, giving the target distribution; [news] bullet 密集预热阶段 (sum, then L1
+    normalisation along the sequence dimension). Reading: the "attention scores" are the
+    softmax weights of each head (logits summed over heads could be negative and have no
+    L1-normalised distribution); the logits are those of the MQA-mode attention, all
+    d_qk dims of the shared latent row, scaled by tau.
+
+    q_t: [H, d_qk]; kv_rows: [m, d_qk] (m >= 1)  ->  [m], summing to 1
+    """
+    z = tau * (q_t @ kv_rows.T)               # [H, m]
+    e = np.exp(z - z.max(axis=1, keepdims=True))
+    a = (e / e.sum(axis=1, keepdims=True)).sum(axis=0)   # sum over heads of each head's weights
+    return a / np.abs(a).sum()                # L1 normalisation along the sequence
+
+
+def indexer_kl(p: np.ndarray, scores: np.ndarray) -> float:
+    """KL(p || softmax(scores)) = sum_s p[s] * (ln p[s] - ln softmax(scores)[s]), 0 ln 0 = 0.
+
+    [blog] section "訓練", Step 1: a KL-divergence loss between the target distribution and
+    the indexer's output is the indexer's training objective; the indexer's distribution is
+    the softmax of its index scores over the same positions. [news] bullet 密集预热阶段
+    (KL散度损失). Natural logarithm.
+    """
+    m = scores.max()
+    log_q = scores - (m + np.log(np.exp(scores - m).sum()))
+    nz = p > 0
+    return float(np.sum(p[nz] * (np.log(p[nz]) - log_q[nz])))
+
+
+def indexer_kl_row(q_bits, kv_bits, idx, index_scores_sel, tau: float) -> float:
+    """The loss term of one query over the positions in ``idx`` (entries < 0 are padding).
+
+    Sparse training stage: [blog] section "訓練", Step 2, and [news] bullet 稀疏训练阶段 --
+    the indexer stays aligned with the main attention distribution, but only over the
+    selected token set S_t. Readings: in that stage the main attention attends to S_t only,
+    so its per-head weights are the softmax over S_t (the weights the sparse attention
+    uses), and the indexer's distribution is the softmax of its scores over S_t. Passing all
+    positions 0..t as ``idx`` gives the dense warm-up term. ``index_scores_sel[j]`` is the
+    index score of position idx[j] (same order; padding entries ignored). With no valid
+    position the term is 0.
+    """
+    idx = np.asarray(idx, dtype=np.int64)
+    keep = idx >= 0
+    sel = idx[keep]
+    if sel.size == 0:
+        return 0.0
+    p = attention_head_sum_target(decode_bf16(q_bits), decode_bf16(kv_bits[sel]), tau)
+    return indexer_kl(p, np.asarray(index_scores_sel, dtype=np.float64)[keep])

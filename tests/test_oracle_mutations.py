@@ -100,8 +100,43 @@ MUTANTS_DRIVER = {
         lambda kc, ks, qs, pos: od.decode_e4m3(kc[: pos + 1], np.full(pos + 1, qs))),
 }
 
+def _target_logits_summed(q, kv, tau):
+    z = (tau * (q @ kv.T)).sum(0)                 # heads summed before the softmax
+    e = np.exp(z - z.max())
+    return e / e.sum()
+
+
+def _target_unnormalised_heads(q, kv, tau):
+    z = tau * (q @ kv.T)
+    a = np.exp(z - z.max()).sum(0)                # no per-head softmax normalisation
+    return a / a.sum()
+
+
+def _kl_reversed(p, scores):
+    q = np.exp(scores - scores.max())
+    q /= q.sum()
+    nz = q > 0
+    return float(np.sum(q[nz] * (np.log(q[nz]) - np.log(np.maximum(p[nz], 1e-300)))))
+
+
+def _kl_log2(p, scores):
+    return od.__dict__["_orig_kl"](p, scores) / np.log(2.0)
+
+
+def _kl_row_keeps_padding(q_bits, kv_bits, idx, sc, tau):
+    idx = np.asarray(idx, dtype=np.int64)
+    sel = np.where(idx >= 0, idx, 0)
+    p = od.attention_head_sum_target(od.decode_bf16(q_bits), od.decode_bf16(kv_bits[sel]), tau)
+    return od.indexer_kl(p, np.asarray(sc, dtype=np.float64))
+
+
 MUTANTS = {
     **{n: ("indexer_topk_row", f) for n, f in MUTANTS_DRIVER.items()},
+    "target_logits_summed_over_heads": ("attention_head_sum_target", _target_logits_summed),
+    "target_heads_not_normalised": ("attention_head_sum_target", _target_unnormalised_heads),
+    "kl_reversed": ("indexer_kl", _kl_reversed),
+    "kl_in_bits": ("indexer_kl", _kl_log2),
+    "kl_row_keeps_padding": ("indexer_kl_row", _kl_row_keeps_padding),
     "relu_after_sum": ("index_scores", _relu_after_sum),
     "no_relu": ("index_scores", _no_relu),
     "unweighted_heads": ("index_scores", _unweighted),
@@ -140,6 +175,7 @@ def test_pins_catch_planted_mistake(mutant, monkeypatch):
     name, fake = MUTANTS[mutant]
     monkeypatch.setitem(od.__dict__, "_orig_attn", od.sparse_mla_attention)
     monkeypatch.setitem(od.__dict__, "_orig_e4m3", od.decode_e4m3)
+    monkeypatch.setitem(od.__dict__, "_orig_kl", od.indexer_kl)
     monkeypatch.setattr(od, name, fake)
     monkeypatch.setattr(oracle, name, fake)
     assert _run_pins(), f"no pin caught mutant {mutant}"

@@ -261,3 +261,110 @@ def test_page_constants_fix_128k_as_131072_and_k_2048():
     assert synthetic.config("prefill_128k").max_len == 131072
     for name in ["prefill_4k", "prefill_32k", "prefill_128k", "decode"]:
         assert synthetic.config(name).topk == g["topk"]["value"]
+
+
+# ----------------------------------------------------------------------------- indexer alignment loss
+def test_head_sum_target_brute_force():
+    # a[s] = sum_h softmax_s(tau q_h . kv_s), p = a / sum(a): explicit loops with math.exp
+    H, m, d = 4, 7, 5
+    q = rng.standard_normal((H, d)) * 2.0
+    kv = rng.standard_normal((m, d))
+    tau = 0.61
+    a = [0.0] * m
+    for h in range(H):
+        z = [tau * sum(q[h, e] * kv[s, e] for e in range(d)) for s in range(m)]
+        zmax = max(z)
+        ex = [math.exp(v - zmax) for v in z]
+        tot = sum(ex)
+        for s in range(m):
+            a[s] += ex[s] / tot
+    expect = [x / sum(a) for x in a]
+    np.testing.assert_allclose(oracle.attention_head_sum_target(q, kv, tau), expect, rtol=1e-12)
+    assert abs(sum(a) - H) < 1e-12                   # each head's weights sum to one
+
+
+def test_head_sum_target_single_head_is_softmax():
+    from scipy.special import softmax
+    q = rng.standard_normal((1, 6))
+    kv = rng.standard_normal((9, 6))
+    np.testing.assert_allclose(oracle.attention_head_sum_target(q, kv, 0.4), softmax(0.4 * (kv @ q[0])), rtol=1e-12)
+
+
+def test_indexer_kl_matches_scipy_entropy():
+    from scipy.special import softmax
+    from scipy.stats import entropy
+    for m in (1, 2, 17, 300):
+        p = rng.random(m) ** 3
+        p /= p.sum()
+        scores = rng.standard_normal(m) * 4.0
+        assert oracle.indexer_kl(p, scores) == pytest.approx(entropy(p, softmax(scores)), rel=1e-11, abs=1e-13)
+
+
+def test_indexer_kl_closed_forms():
+    p = rng.random(11)
+    p /= p.sum()
+    assert abs(oracle.indexer_kl(p, np.log(p) + 3.7)) < 1e-13          # scores = ln p + c: zero
+    assert oracle.indexer_kl(np.full(5, 0.2), np.full(5, -2.5)) == pytest.approx(0.0, abs=1e-15)
+    x, y, a = 1.3, -0.4, 0.3                                           # two points
+    sig = 1.0 / (1.0 + math.exp(-(x - y)))
+    two = a * math.log(a / sig) + (1 - a) * math.log((1 - a) / (1 - sig))
+    assert oracle.indexer_kl(np.array([a, 1 - a]), np.array([x, y])) == pytest.approx(two, rel=1e-13)
+    s = rng.standard_normal(6)                                         # one-hot target: -ln q_0
+    lse = math.log(sum(math.exp(v) for v in s))
+    assert oracle.indexer_kl(np.eye(6)[0], s) == pytest.approx(lse - s[0], rel=1e-13)
+
+
+def test_indexer_kl_is_nonnegative():
+    for _ in range(50):
+        m = int(rng.integers(1, 40))
+        p = rng.random(m)
+        p /= p.sum()
+        assert oracle.indexer_kl(p, rng.standard_normal(m) * 3.0) >= -1e-15
+
+
+def _kl_row_inputs(H=3, n=12, d=8):
+    qb = torch.tensor(rng.standard_normal((H, d)), dtype=torch.float32).to(torch.bfloat16)
+    kvb = torch.tensor(rng.standard_normal((n, d)), dtype=torch.float32).to(torch.bfloat16)
+    u16 = lambda t: t.view(torch.int16).numpy().view(np.uint16)           # noqa: E731
+    return u16(qb), u16(kvb), qb.double().numpy(), kvb.double().numpy()
+
+
+def test_indexer_kl_row_brute_force_over_the_selected_set():
+    # sparse stage: per-head softmax over the selected rows only, head sum, L1 normalisation,
+    # KL against the softmax of the selected rows' index scores -- all with explicit loops
+    qb, kvb, q, kv = _kl_row_inputs()
+    H, d = q.shape
+    idx = [7, 2, 9, 4, 11]
+    sc = rng.standard_normal(len(idx)) * 2.0
+    tau = 0.35
+    a = [0.0] * len(idx)
+    for h in range(H):
+        z = [tau * sum(q[h, e] * kv[s, e] for e in range(d)) for s in idx]
+        ex = [math.exp(v) for v in z]
+        for j in range(len(idx)):
+            a[j] += ex[j] / sum(ex)
+    p = [x / sum(a) for x in a]
+    lse = math.log(sum(math.exp(v) for v in sc))
+    expect = sum(p[j] * (math.log(p[j]) - (sc[j] - lse)) for j in range(len(idx)))
+    assert oracle.indexer_kl_row(qb, kvb, idx, sc, tau) == pytest.approx(expect, rel=1e-12)
+
+
+def test_indexer_kl_row_ignores_padding_and_order():
+    qb, kvb, _, _ = _kl_row_inputs()
+    idx = np.array([3, 8, 0, 5])
+    sc = rng.standard_normal(4)
+    base = oracle.indexer_kl_row(qb, kvb, idx, sc, 0.5)
+    perm = np.array([2, 0, 3, 1])
+    padded_idx = np.array([-1, 3, -1, 8, 0, -1, 5])
+    padded_sc = np.array([9.0, sc[0], -7.0, sc[1], sc[2], 5.0, sc[3]])
+    assert oracle.indexer_kl_row(qb, kvb, idx[perm], sc[perm], 0.5) == pytest.approx(base, rel=1e-12)
+    assert oracle.indexer_kl_row(qb, kvb, padded_idx, padded_sc, 0.5) == pytest.approx(base, rel=1e-12)
+    assert oracle.indexer_kl_row(qb, kvb, [-1, -1], [0.0, 1.0], 0.5) == 0.0
+
+
+def test_head_sum_target_matches_attention_weights_from_lse():
+    # p[s] = (1/H) sum_h exp(tau q_h . kv_s - lse_h), lse from the attention oracle
+    qb, kvb, q, kv = _kl_row_inputs(H=5, n=9)
+    _, lse = oracle.sparse_mla_attention(q, kv, 4, 0.3)
+    a = np.exp(0.3 * (q @ kv.T) - lse[:, None]).sum(0) / q.shape[0]
+    np.testing.assert_allclose(oracle.attention_head_sum_target(q, kv, 0.3), a, rtol=1e-12)
