@@ -203,7 +203,7 @@ def test_attention_weights_sum_to_one_and_lse_is_logsumexp():
     kv[:, :dv] = 1.0                                   # V = ones  =>  out = sum_s p_s = 1
     out, lse = oracle.sparse_mla_attention(q, kv, dv, 0.7)
     np.testing.assert_allclose(out, 1.0, rtol=1e-13)
-    np.testing.assert_allclose(lse, logsumexp(0.7 * q @ kv.T, axis=1), rtol=1e-13)
+    np.testing.assert_allclose(lse, logsumexp(0.7 * q @ kv.T, axis=1), rtol=1e-13, atol=1e-13)
 
 
 def test_attention_closed_forms():
