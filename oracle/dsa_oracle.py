@@ -35,7 +35,9 @@ one-row and equal-logit closed forms and to scipy's logsumexp; the
 indexer-alignment loss to explicit loops (per-head softmax, head sum, L1
 normalisation, KL), to scipy's softmax and relative entropy, to its closed forms
 (zero for scores = ln p + c, two points, one-hot) and to Gibbs' inequality, and
-its per-query term to padding and order invariance. Absolute values
+its per-query term to padding and order invariance; the masked dense mode to
+torch's scaled_dot_product_attention in float64 with a boolean mask and to the
+sparse attention over the unmasked rows. Absolute values
 at the production shapes have no printed example on the pages: beyond these
 invariants and reductions they are parity-unpinned by the pages.
 """
@@ -46,7 +48,7 @@ import numpy as np
 __all__ = [
     "decode_e4m3", "decode_bf16", "index_scores", "select_topk", "sparse_mla_attention",
     "indexer_topk_row", "sparse_mla_attn_row", "dsa_row",
-    "attention_head_sum_target", "indexer_kl", "indexer_kl_row",
+    "attention_head_sum_target", "indexer_kl", "indexer_kl_row", "masked_dense_mqa_attention",
 ]
 
 
@@ -241,3 +243,29 @@ def indexer_kl_row(q_bits, kv_bits, idx, index_scores_sel, tau: float) -> float:
         return 0.0
     p = attention_head_sum_target(decode_bf16(q_bits), decode_bf16(kv_bits[sel]), tau)
     return indexer_kl(p, np.asarray(index_scores_sel, dtype=np.float64)[keep])
+
+
+# ----------------------------------------------------------------------------- masked dense mode
+def masked_dense_mqa_attention(q_t: np.ndarray, kv_prefix: np.ndarray, mask: np.ndarray, d_v: int, tau: float):
+    """Dense attention of one query over every row of ``kv_prefix`` (positions 0..pos), with the
+    logits of rows where ``mask`` is False set to -inf before the softmax.
+
+    [news] bullet 实际服务部署: for short-sequence prefill the deployment uses a masked mode that
+    emulates the effect of DSA. Reading: the mask is the top-k selection of the query, so the
+    result equals the attention over the selected rows (MQA mode, as in
+    ``sparse_mla_attention``), computed densely over the causal prefix. With no row unmasked:
+    out = 0, lse = -inf.
+
+    q_t: [H, d_qk]; kv_prefix: [pos+1, d_qk]; mask: [pos+1] bool  ->  out [H, d_v], lse [H]
+    """
+    H = q_t.shape[0]
+    mask = np.asarray(mask, dtype=bool)
+    if not mask.any():
+        return np.zeros((H, d_v)), np.full(H, -np.inf)
+    z = tau * (q_t @ kv_prefix.T)             # [H, pos+1], every causal row
+    z = np.where(mask[None, :], z, -np.inf)
+    zmax = z.max(axis=1)
+    e = np.exp(z - zmax[:, None])             # exp(-inf) = 0 for masked rows
+    l = e.sum(axis=1)
+    out = (e @ kv_prefix[:, :d_v]) / l[:, None]
+    return out, zmax + np.log(l)

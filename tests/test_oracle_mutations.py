@@ -130,8 +130,20 @@ def _kl_row_keeps_padding(q_bits, kv_bits, idx, sc, tau):
     return od.indexer_kl(p, np.asarray(sc, dtype=np.float64))
 
 
+def _masked_ignores_mask(q, kv, mask, d_v, tau):
+    return od.sparse_mla_attention(q, kv, d_v, tau)
+
+
+def _masked_zero_logits(q, kv, mask, d_v, tau):
+    z = np.where(np.asarray(mask)[None, :], tau * (q @ kv.T), 0.0)     # masked logits 0, not -inf
+    e = np.exp(z - z.max(1, keepdims=True))
+    return (e @ kv[:, :d_v]) / e.sum(1, keepdims=True), z.max(1) + np.log(e.sum(1))
+
+
 MUTANTS = {
     **{n: ("indexer_topk_row", f) for n, f in MUTANTS_DRIVER.items()},
+    "masked_mode_ignores_mask": ("masked_dense_mqa_attention", _masked_ignores_mask),
+    "masked_logits_zero_not_minus_inf": ("masked_dense_mqa_attention", _masked_zero_logits),
     "target_logits_summed_over_heads": ("attention_head_sum_target", _target_logits_summed),
     "target_heads_not_normalised": ("attention_head_sum_target", _target_unnormalised_heads),
     "kl_reversed": ("indexer_kl", _kl_reversed),

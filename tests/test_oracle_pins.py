@@ -368,3 +368,37 @@ def test_head_sum_target_matches_attention_weights_from_lse():
     _, lse = oracle.sparse_mla_attention(q, kv, 4, 0.3)
     a = np.exp(0.3 * (q @ kv.T) - lse[:, None]).sum(0) / q.shape[0]
     np.testing.assert_allclose(oracle.attention_head_sum_target(q, kv, 0.3), a, rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------- masked dense mode
+def test_masked_dense_attention_matches_sdpa_with_a_boolean_mask():
+    # every query of a short causal prefill, its mask a random subset of 0..t (never empty):
+    # torch scaled_dot_product_attention in float64 with the mask as attn_mask
+    L, H, dqk, dv = 23, 3, 10, 6
+    q = rng.standard_normal((L, H, dqk))
+    kv = rng.standard_normal((L, dqk))
+    tau = 0.37
+    masks = np.tril(rng.random((L, L)) < 0.6)
+    masks[np.arange(L), rng.integers(0, np.arange(L) + 1)] = True
+    qt = torch.from_numpy(q).permute(1, 0, 2)[None]
+    kt = torch.from_numpy(kv)[None, None].expand(1, H, L, dqk)
+    vt = torch.from_numpy(kv[:, :dv])[None, None].expand(1, H, L, dv)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=torch.from_numpy(masks), scale=tau)
+    ref = ref[0].permute(1, 0, 2).numpy()
+    for t in range(L):
+        out, _ = oracle.masked_dense_mqa_attention(q[t], kv[: t + 1], masks[t, : t + 1], dv, tau)
+        np.testing.assert_allclose(out, ref[t], rtol=1e-11, atol=1e-12)
+
+
+def test_masked_dense_attention_equals_sparse_attention_over_the_mask():
+    H, n, dqk, dv = 4, 30, 8, 5
+    q = rng.standard_normal((H, dqk)) * 2.0
+    kv = rng.standard_normal((n, dqk))
+    mask = rng.random(n) < 0.3
+    mask[7] = True
+    out_d, lse_d = oracle.masked_dense_mqa_attention(q, kv, mask, dv, 0.45)
+    out_s, lse_s = oracle.sparse_mla_attention(q, kv[mask], dv, 0.45)
+    np.testing.assert_allclose(out_d, out_s, rtol=1e-12)
+    np.testing.assert_allclose(lse_d, lse_s, rtol=1e-12)
+    out_e, lse_e = oracle.masked_dense_mqa_attention(q, kv, np.zeros(n, dtype=bool), dv, 0.45)
+    assert (out_e == 0).all() and np.isneginf(lse_e).all()
