@@ -279,13 +279,29 @@ def run_ours(args, cfg, rank, world, local_rank):
     seed = rank_seed(args.seed, rank)
     do_idx = args.stage in ("all", "indexer")
     do_att = args.stage in ("all", "attention")
-    q_idx, q_scale = synthetic.gen_q_idx(cfg, seed, dev)
+    do_loss = args.with_loss
+    attn_fn = dsa.dsa_masked_mqa_attn if args.attn_mode == "masked" else dsa.dsa_sparse_mla_attn
     k_idx, k_scale = synthetic.gen_k_idx(cfg, seed, dev)
-    g = {"q_idx": q_idx, "k_idx": k_idx, "w": synthetic.gen_w(cfg, seed, dev),
-         "lengths": synthetic.lengths(cfg, seed).to(dev)}
-    if do_att:
-        g["q"] = synthetic.gen_q(cfg, seed, dev)
-        g["kv"] = synthetic.gen_kv(cfg, seed, dev)
+    if args.chunk_queries:
+        # the call for the last C queries of one sequence (n_q = C over the whole key side), as the
+        # chunked and row-sharded runs make it; for profiling a long context at a small footprint
+        import dataclasses
+        toks = range(cfg.max_len - args.chunk_queries, cfg.max_len)
+        cfg = dataclasses.replace(cfg, n_q=args.chunk_queries)
+        q_idx, q_scale = synthetic.gen_q_idx(cfg, seed, dev, tokens=toks)
+        g = {"q_idx": q_idx.view(1, cfg.n_q, cfg.n_idx_heads, cfg.idx_dim), "k_idx": k_idx,
+             "w": synthetic.gen_w(cfg, seed, dev, tokens=toks).view(1, cfg.n_q, -1),
+             "lengths": synthetic.lengths(cfg, seed).to(dev)}
+        if do_att:
+            g["q"] = synthetic.gen_q(cfg, seed, dev, tokens=toks).view(1, cfg.n_q, cfg.n_heads, cfg.d_qk)
+            g["kv"] = synthetic.gen_kv(cfg, seed, dev)
+    else:
+        q_idx, q_scale = synthetic.gen_q_idx(cfg, seed, dev)
+        g = {"q_idx": q_idx, "k_idx": k_idx, "w": synthetic.gen_w(cfg, seed, dev),
+             "lengths": synthetic.lengths(cfg, seed).to(dev)}
+        if do_att:
+            g["q"] = synthetic.gen_q(cfg, seed, dev)
+            g["kv"] = synthetic.gen_kv(cfg, seed, dev)
     scales = torch.cat([q_scale.reshape(-1), k_scale.reshape(-1)]).contiguous()
     dims = dsa.dims_for(cfg)
     ws = dsa.Workspace.create(dims, cfg.topk, device=dev)
@@ -293,6 +309,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     if do_att:
         out = torch.empty((cfg.batch, cfg.n_q, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
         lse = torch.empty((cfg.batch, cfg.n_q, cfg.n_heads), dtype=torch.float32, device=dev)
+    idx_scores = torch.empty((cfg.batch, cfg.n_q, cfg.topk), dtype=torch.float32, device=dev) if do_loss else None
+    loss = torch.empty((cfg.batch, cfg.n_q), dtype=torch.float32, device=dev) if do_loss else None
     stream = torch.cuda.current_stream(dev)
 
     if not do_idx:   # the attention still needs real selections: compute them once, untimed
@@ -302,15 +320,22 @@ def run_ours(args, cfg, rank, world, local_rank):
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        if do_idx:
+        if do_idx and do_loss:       # the selection with the index score of every selected entry
+            dsa.dsa_indexer_topk_scores(dims, g["q_idx"], g["w"], g["k_idx"], scales, g["lengths"], cfg.topk, idx,
+                                        idx_scores, ws.buf, stream)
+        elif do_idx:
             dsa.dsa_indexer_topk(dims, g["q_idx"], g["w"], g["k_idx"], scales, g["lengths"], cfg.topk, idx, ws.buf,
                                  stream)
         if ev is not None:
             ev[1].record(stream)
         if do_att:
-            dsa.dsa_sparse_mla_attn(dims, g["q"], g["kv"], idx, cfg.topk, out, lse, ws.buf, stream)
+            attn_fn(dims, g["q"], g["kv"], idx, cfg.topk, out, lse, ws.buf, stream)
         if ev is not None:
             ev[2].record(stream)
+        if do_loss:
+            dsa.dsa_indexer_kl_loss(dims, g["q"], g["kv"], idx, idx_scores, lse, cfg.topk, loss, ws.buf, stream)
+        if ev is not None:
+            ev[3].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -322,7 +347,7 @@ def run_ours(args, cfg, rank, world, local_rank):
             torch.distributed.barrier()
         torch.cuda.synchronize(dev)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     sampler = ClockSampler(local_rank) if rank == 0 else None
     barrier()
     start = torch.cuda.Event(enable_timing=True)
@@ -337,6 +362,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     total_ms = start.elapsed_time(end)
     idx_ms = [e[0].elapsed_time(e[1]) for e in evs]
     att_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    loss_ms = [e[2].elapsed_time(e[3]) for e in evs] if do_loss else None
     total_ms = max_over_ranks(total_ms, dev)
 
     # ---------------- end to end through the public API with host buffers
@@ -347,8 +373,15 @@ def run_ours(args, cfg, rank, world, local_rank):
     # dims other than the production ones add the copies into padded layouts (3 before the
     # indexer; 2 before and 2 after the attention)
     padded = (cfg.n_idx_heads, cfg.idx_dim, cfg.n_heads, cfg.d_latent, cfg.d_rope) != (64, 128, 128, 512, 64)
-    launches = ((2 if cfg.is_decode else 1) + (3 if padded else 0)) * int(do_idx) + (1 + (4 if padded else 0)) * int(do_att)
-    return dict(total_ms=total_ms, idx_ms=idx_ms, att_ms=att_ms, clocks=clocks, e2e=e2e, launches_per_step=launches)
+    # a prefill whose items reach the indexer's sampled threshold adds its exact pass (a second
+    # launch of the same kernel over the items, if any, whose sampled threshold failed)
+    sampled = (not cfg.is_decode) and cfg.topk >= 1024 and cfg.max_len >= 64 * 128
+    idx_launches = 2 if cfg.is_decode else (2 if sampled else 1)
+    att_launches = (2 if args.attn_mode == "masked" else 1) + (4 if padded else 0)     # masked: bitmap kernel
+    launches = ((idx_launches + (3 if padded else 0)) * int(do_idx) + att_launches * int(do_att) +
+                (1 + (2 if padded else 0)) * int(do_loss))
+    return dict(total_ms=total_ms, idx_ms=idx_ms, att_ms=att_ms, loss_ms=loss_ms, clocks=clocks, e2e=e2e,
+                launches_per_step=launches)
 
 
 
@@ -669,6 +702,18 @@ def run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
             "chunk_queries": C, "streams": "h2d / compute / d2h overlapped"}
 
 
+def torchrun_command(n: int, argv, port: int):
+    """The command that runs bench.py with ``argv`` as n ranks on this node (127.0.0.1)."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+
+
+def relaunch_under_torchrun(n: int, argv) -> int:
+    cmd = torchrun_command(n, argv, _free_port())
+    # the ranks' process group times out well before this last bound
+    return subprocess.call(["timeout", "-k", "60", "3600", *cmd])
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -678,7 +723,9 @@ def main():
     ap.add_argument("--workload", default="prefill_128k", choices=["tiny", "prefill_4k", "prefill_32k", "prefill_128k", "decode"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--print-ranks", action="store_true",
+                    help="print each rank's RANK/LOCAL_RANK/WORLD_SIZE as JSON and exit (checks the launch)")
     ap.add_argument("--e2e-chunk", type=int, default=4096,
                     help="queries per dsa_forward call in the e2e measurement (0 = one call per step)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -687,10 +734,24 @@ def main():
     ap.add_argument("--stage", default="all", choices=["all", "indexer", "attention"],
                     help="time one stage only (profiling); the line then reports that stage")
     ap.add_argument("--seq-len", type=int, default=0, help="override L of a prefill workload (profiling)")
+    ap.add_argument("--chunk-queries", type=int, default=0,
+                    help="prefill: time the call for the last N queries only (profiling a long context small)")
+    ap.add_argument("--attn-mode", default="sparse", choices=["sparse", "masked"],
+                    help="attention stage: the sparse kernel, or the masked dense mode (max_len <= 16384)")
+    ap.add_argument("--with-loss", action="store_true",
+                    help="the step also computes the indexer-alignment KL loss (selection with scores, attention, "
+                         "loss)")
     ap.add_argument("--shard", default="sequences", choices=["sequences", "rows"],
                     help="N>1: one sequence per rank (weak scaling), or one sequence's query rows split over "
                          "the ranks with an all-gather of the key-side caches per step (strong scaling)")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: run this same command under torchrun
+        return relaunch_under_torchrun(args.gpus, sys.argv[1:])
+    if args.print_ranks:
+        print(json.dumps({k: os.environ.get(k) for k in ("RANK", "LOCAL_RANK", "WORLD_SIZE", "MASTER_ADDR")}),
+              flush=True)
+        return 0
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     cfg = synthetic.config(args.workload)
@@ -700,7 +761,7 @@ def main():
         import dataclasses
         cfg = dataclasses.replace(cfg, n_q=args.seq_len, max_len=args.seq_len, name=f"prefill_L{args.seq_len}",
                                   description=f"causal prefill L={args.seq_len}, k=2048")
-    if args.stage != "all":
+    if args.stage != "all" or args.with_loss or args.attn_mode != "sparse" or args.chunk_queries:
         args.no_e2e = True
         args.no_cpu_baseline = True
     rank = int(os.environ.get("RANK", "0"))
@@ -736,7 +797,12 @@ def report(args, cfg, res, world):
     peaks = _peaks()
     sh = res.get("shard")
     # row sharding: rank 0's rows set the per-stage work (the job's time is the slowest rank's)
-    w = _work_rows(cfg, *sh["rank0_rows"]) if sh else _work(cfg, rank_seed(args.seed, 0))
+    if sh:
+        w = _work_rows(cfg, *sh["rank0_rows"])
+    elif getattr(args, "chunk_queries", 0):
+        w = _work_rows(cfg, cfg.max_len - args.chunk_queries, cfg.max_len)
+    else:
+        w = _work(cfg, rank_seed(args.seed, 0))
     metric, unit = _metric(cfg)
     ms_step = res["total_ms"] / args.steps
     idx_ms = statistics.mean(res["idx_ms"])
@@ -769,6 +835,18 @@ def report(args, cfg, res, world):
                                          "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
                                          "peak_note": f"{peaks['source']} sustained bf16",
                                          "gather_GBps": w["attn_gather_bytes"] / (att_ms / 1e3) / 1e9}
+            if getattr(args, "attn_mode", "sparse") == "masked":
+                stages["sparse_mla_attn"]["mode"] = ("masked dense (whole 64-row blocks of each causal prefix; "
+                                                     "work counted over the selected rows only)")
+    if res.get("loss_ms"):
+        # indexer-alignment loss: the logits of every selected row again (2 x 128 heads x 576 dims per row)
+        # plus the gather of its latent row; bf16 tensor-bound in principle, like the attention's logits half
+        loss_ms = statistics.mean(res["loss_ms"])
+        stages["indexer_kl_loss"] = {"ms": loss_ms, "bound": "tensor",
+                                     "achieved": w["sel_rows"] * 2 * cfg.n_heads * cfg.d_qk / (loss_ms / 1e3) / 1e12,
+                                     "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                                     "peak_note": f"{peaks['source']} sustained bf16",
+                                     "gather_GBps": w["attn_gather_bytes"] / (loss_ms / 1e3) / 1e9}
     for k, st in stages.items():
         st["frac"] = st["achieved"] / st["peak"]
     dom = max(stages, key=lambda k: stages[k]["ms"])
@@ -802,7 +880,10 @@ def report(args, cfg, res, world):
         stages["allgather"] = {"ms": statistics.mean(res["gather_ms"]), "bytes": key_bytes,
                                "note": "rank 0's view; every rank receives the whole key side"}
     else:
-        value = aggregate_value(cfg.batch * cfg.n_q, args.steps, world, res["total_ms"])
+        n_tok = getattr(args, "chunk_queries", 0) or cfg.batch * cfg.n_q
+        value = aggregate_value(n_tok, args.steps, world, res["total_ms"])
+        if getattr(args, "chunk_queries", 0):
+            conf["workload"] += f" -- the call for its last {args.chunk_queries} queries only"
     line = {
         "metric": metric, "value": value,
         "unit": unit,

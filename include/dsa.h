@@ -94,6 +94,17 @@ dsa_status dsa_indexer_topk(const dsa_dims* dims, const void* q_idx, const void*
                             void* ws, size_t ws_bytes, dsa_stream_t stream);
 
 /*
+ * dsa_indexer_topk that also returns the index score of every selected position:
+ *   out_scores fp32 [B, n_q, topk]  out_scores[b,i,j] = I[t, out_idx[b,i,j]] as the kernel computed
+ *              it in fp32 from the decoded inputs (scales applied); -inf where out_idx is -1.
+ * out_scores may be NULL (then identical to dsa_indexer_topk). The scores feed the indexer's
+ * alignment loss (dsa_indexer_kl_loss).
+ */
+dsa_status dsa_indexer_topk_scores(const dsa_dims* dims, const void* q_idx, const void* w, const void* k_idx,
+                                   const float* scales, const int32_t* lengths, int32_t topk, int32_t* out_idx,
+                                   float* out_scores, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/*
  * Stage 3: sparse MLA attention (MQA mode) over the selected rows.
  *   q         bf16  [B, n_q, n_heads, d_latent + d_rope]  (16-byte aligned)
  *   latent_kv bf16  [B, max_len, d_latent + d_rope]       (16-byte aligned) one row per token
@@ -108,6 +119,43 @@ dsa_status dsa_indexer_topk(const dsa_dims* dims, const void* q_idx, const void*
 dsa_status dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void* latent_kv, const int32_t* idx,
                                int32_t topk, void* out, float* lse, void* ws, size_t ws_bytes,
                                dsa_stream_t stream);
+
+/*
+ * Stage 3 in the masked dense mode, for short prefill: the same result as dsa_sparse_mla_attn
+ * (same arguments and layouts), computed as dense attention of each query over its positions
+ * 0 .. e-1 (e = one past its last valid index) with every position the index row does not
+ * list masked out. "DeepSeek 发布新模型 V3.2-Exp：基于DSA稀疏注意力机制的长上下文优化", bullet
+ * 实际服务部署: short-sequence prefill uses a masked mode that emulates DSA. The key rows are
+ * read as whole 64-row blocks (TMA tile copies) instead of gathered row by row.
+ * Differences from dsa_sparse_mla_attn: a position listed twice is attended once; every latent
+ * row the blocks touch (positions 0 .. 64*ceil(e/64)-1 of the query's sequence) must hold
+ * finite values, since a masked row still enters the weighted sum with weight zero.
+ * Requires max_len <= 16384 (else DSA_ERR_UNSUPPORTED). Uses workspace for one bitmap row per
+ * query (included in dsa_workspace_bytes for such dims).
+ */
+dsa_status dsa_masked_mqa_attn(const dsa_dims* dims, const void* q, const void* latent_kv, const int32_t* idx,
+                               int32_t topk, void* out, float* lse, void* ws, size_t ws_bytes,
+                               dsa_stream_t stream);
+
+/*
+ * Forward of the indexer-alignment loss, one term per query. "節前發版：Deepseek v3.2 exp",
+ * section "訓練", Step 1 / Step 2, and "DeepSeek 发布新模型 V3.2-Exp：...", bullets 密集预热阶段
+ * / 稀疏训练阶段: the target distribution sums the main attention over all heads and
+ * L1-normalises it along the sequence; the loss is the KL divergence from it to the softmax of
+ * the index scores, both over the query's selected entries in the sparse stage:
+ *   a_s = sum_h exp(tau * q_h . kv_s - lse_h),  p_s = a_s / sum_s a_s,
+ *   loss[t] = sum_s p_s * (ln p_s - ln softmax_s(I_s))          (natural log)
+ * over the valid entries s of idx[t] (< 0 padding; >= max_len reported as DSA_ERR_INDEX_RANGE
+ * and skipped). Passing every position 0..t of a query (topk >= t+1) gives the dense warm-up term.
+ *   q, latent_kv, idx  as for dsa_sparse_mla_attn
+ *   idx_scores  fp32 [B, n_q, topk]  the index score of each entry (dsa_indexer_topk_scores)
+ *   lse         fp32 [B, n_q, n_heads]  the lse output of dsa_sparse_mla_attn on the same idx
+ *   loss        fp32 [B, n_q]  the per-query term (0 for a query with no valid entry); the
+ *               training objective is its sum over the queries.
+ */
+dsa_status dsa_indexer_kl_loss(const dsa_dims* dims, const void* q, const void* latent_kv, const int32_t* idx,
+                               const float* idx_scores, const float* lse, int32_t topk, float* loss, void* ws,
+                               size_t ws_bytes, dsa_stream_t stream);
 
 /*
  * The whole forward path: dsa_indexer_topk then dsa_sparse_mla_attn on the same stream.
@@ -147,6 +195,16 @@ dsa_status dsa_indexer_topk_decode_noalloc(const dsa_dims* dims, const void* q_i
 /* Synchronises `stream`, returns the first device-side error recorded in `ws` since the
  * last call (DSA_OK if none) and clears it. `detail`, if non-NULL, receives a location tag. */
 dsa_status dsa_get_device_status(void* ws, dsa_stream_t stream, uint32_t* detail);
+
+/*
+ * Test setting for failure detection: the time budget of every bounded wait in the indexer's
+ * pipeline (dsa_indexer_topk*, forward's first stage), in ns; 0 restores the default of 2 s.
+ * Process-wide, read at each launch. With a budget too short for the pipeline's handshakes a
+ * launch stops early: its waits record DSA_ERR_DEVICE_TIMEOUT in the status word, every role
+ * ends, the teardown still lets in-flight copies and MMAs land (under their own fixed budget),
+ * and the selection written is incomplete. Not for production use.
+ */
+dsa_status dsa_set_wait_budget_ns(uint64_t ns);
 
 /* Static description of a status code. Never NULL. */
 const char* dsa_status_string(dsa_status status);

@@ -31,7 +31,8 @@ DSA_ERR_DEVICE_TIMEOUT, DSA_ERR_INDEX_RANGE, DSA_ERR_WORKSPACE = 4, 5, 6
 LIBRARY_PATH = _LIB_PATH
 EXPORTED = ("dsa_workspace_bytes", "dsa_workspace_init", "dsa_indexer_topk", "dsa_sparse_mla_attn",
             "dsa_forward", "dsa_get_device_status", "dsa_status_string", "dsa_version",
-            "dsa_indexer_topk_decode_noalloc")
+            "dsa_indexer_topk_decode_noalloc", "dsa_masked_mqa_attn", "dsa_indexer_topk_scores",
+            "dsa_indexer_kl_loss", "dsa_set_wait_budget_ns")
 
 
 class dsa_dims(ctypes.Structure):
@@ -48,14 +49,22 @@ _lib.dsa_workspace_init.argtypes = [_P, ctypes.c_size_t, _P]
 _lib.dsa_workspace_init.restype = ctypes.c_int
 _lib.dsa_indexer_topk.argtypes = [_DIMS, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]
 _lib.dsa_indexer_topk.restype = ctypes.c_int
+_lib.dsa_indexer_topk_scores.argtypes = [_DIMS, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.dsa_indexer_topk_scores.restype = ctypes.c_int
+_lib.dsa_indexer_kl_loss.argtypes = [_DIMS, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]
+_lib.dsa_indexer_kl_loss.restype = ctypes.c_int
 _lib.dsa_sparse_mla_attn.argtypes = [_DIMS, _P, _P, _P, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.dsa_sparse_mla_attn.restype = ctypes.c_int
+_lib.dsa_masked_mqa_attn.argtypes = [_DIMS, _P, _P, _P, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.dsa_masked_mqa_attn.restype = ctypes.c_int
 _lib.dsa_forward.argtypes = [_DIMS, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.dsa_forward.restype = ctypes.c_int
 _lib.dsa_get_device_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
 _lib.dsa_get_device_status.restype = ctypes.c_int
 _lib.dsa_status_string.argtypes = [ctypes.c_int]
 _lib.dsa_status_string.restype = ctypes.c_char_p
+_lib.dsa_set_wait_budget_ns.argtypes = [ctypes.c_uint64]
+_lib.dsa_set_wait_budget_ns.restype = ctypes.c_int
 _lib.dsa_version.argtypes = []
 _lib.dsa_version.restype = ctypes.c_int32
 
@@ -68,6 +77,11 @@ class DSAError(RuntimeError):
 
 def dsa_status_string(status: int) -> str:
     return _lib.dsa_status_string(int(status)).decode()
+
+
+def dsa_set_wait_budget_ns(ns: int):
+    """Test setting: budget of the indexer's pipeline waits in ns (0 = the default 2 s)."""
+    _check(_lib.dsa_set_wait_budget_ns(int(ns)), "dsa_set_wait_budget_ns")
 
 
 def dsa_version() -> int:
@@ -122,9 +136,26 @@ def dsa_indexer_topk(dims, q_idx, w, k_idx, scales, lengths, topk, out_idx, ws, 
            "dsa_indexer_topk")
 
 
+def dsa_indexer_topk_scores(dims, q_idx, w, k_idx, scales, lengths, topk, out_idx, out_scores, ws, stream=None):
+    _check(_lib.dsa_indexer_topk_scores(ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(scales),
+                                        _ptr(lengths), int(topk), _ptr(out_idx), _ptr(out_scores), _ptr(ws),
+                                        ws.numel(), _stream(stream)), "dsa_indexer_topk_scores")
+
+
+def dsa_indexer_kl_loss(dims, q, latent_kv, idx, idx_scores, lse, topk, loss, ws, stream=None):
+    _check(_lib.dsa_indexer_kl_loss(ctypes.byref(dims), _ptr(q), _ptr(latent_kv), _ptr(idx), _ptr(idx_scores),
+                                    _ptr(lse), int(topk), _ptr(loss), _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_indexer_kl_loss")
+
+
 def dsa_sparse_mla_attn(dims, q, latent_kv, idx, topk, out, lse, ws, stream=None):
     _check(_lib.dsa_sparse_mla_attn(ctypes.byref(dims), _ptr(q), _ptr(latent_kv), _ptr(idx), int(topk), _ptr(out),
                                     _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)), "dsa_sparse_mla_attn")
+
+
+def dsa_masked_mqa_attn(dims, q, latent_kv, idx, topk, out, lse, ws, stream=None):
+    _check(_lib.dsa_masked_mqa_attn(ctypes.byref(dims), _ptr(q), _ptr(latent_kv), _ptr(idx), int(topk), _ptr(out),
+                                    _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)), "dsa_masked_mqa_attn")
 
 
 def dsa_forward(dims, q_idx, w, k_idx, scales, lengths, topk, q, latent_kv, out_idx, out, lse, ws, stream=None):
@@ -187,6 +218,36 @@ def sparse_mla_attn(dims, q, latent_kv, idx, topk, ws: Workspace, stream=None):
     out = torch.empty((dims.batch, dims.n_q, dims.n_heads, dims.d_latent), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((dims.batch, dims.n_q, dims.n_heads), dtype=torch.float32, device=q.device)
     dsa_sparse_mla_attn(dims, q, latent_kv, idx.to(torch.int32).contiguous(), topk, out, lse, ws.buf, stream)
+    return out, lse
+
+
+def indexer_topk_scores(dims, q_idx, w, k_idx, q_scale, k_scale, lengths, topk, ws: Workspace, stream=None):
+    """Returns (idx int32 [B, n_q, topk], scores fp32 [B, n_q, topk]); -1 / -inf padded."""
+    _expect(q_idx, torch.uint8, "q_idx")
+    _expect(k_idx, torch.uint8, "k_idx")
+    _expect(w, torch.bfloat16, "w")
+    out_idx = torch.empty((dims.batch, dims.n_q, topk), dtype=torch.int32, device=q_idx.device)
+    out_scores = torch.empty((dims.batch, dims.n_q, topk), dtype=torch.float32, device=q_idx.device)
+    dsa_indexer_topk_scores(dims, q_idx, w, k_idx, _scales(q_scale, k_scale), lengths.to(torch.int32).contiguous(),
+                            topk, out_idx, out_scores, ws.buf, stream)
+    return out_idx, out_scores
+
+
+def indexer_kl_loss(dims, q, latent_kv, idx, idx_scores, lse, topk, ws: Workspace, stream=None):
+    """Returns the per-query indexer-alignment KL terms, fp32 [B, n_q]."""
+    loss = torch.empty((dims.batch, dims.n_q), dtype=torch.float32, device=q.device)
+    dsa_indexer_kl_loss(dims, q, latent_kv, idx.to(torch.int32).contiguous(), idx_scores.contiguous(),
+                        lse.contiguous(), topk, loss, ws.buf, stream)
+    return loss
+
+
+def masked_mqa_attn(dims, q, latent_kv, idx, topk, ws: Workspace, stream=None):
+    """The masked dense mode of the attention. Returns (out, lse) like ``sparse_mla_attn``."""
+    _expect(q, torch.bfloat16, "q")
+    _expect(latent_kv, torch.bfloat16, "latent_kv")
+    out = torch.empty((dims.batch, dims.n_q, dims.n_heads, dims.d_latent), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((dims.batch, dims.n_q, dims.n_heads), dtype=torch.float32, device=q.device)
+    dsa_masked_mqa_attn(dims, q, latent_kv, idx.to(torch.int32).contiguous(), topk, out, lse, ws.buf, stream)
     return out, lse
 
 

@@ -7,11 +7,13 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "dsa.h"
 #include "indexer_topk.cuh"
 #include "sparse_mla.cuh"
+#include "indexer_kl.cuh"
 
 namespace dsa {
 
@@ -55,6 +57,17 @@ __global__ void unpad_rows_kernel(const T* __restrict__ src, T* __restrict__ dst
   }
 }
 
+// Sets columns [cols_from, cols) of each of `rows` rows of width `cols` to `v`.
+template <typename T>
+__global__ void fill_cols_kernel(T* __restrict__ dst, int64_t rows, int cols_from, int cols, T v) {
+  const int64_t per = cols - cols_from;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < rows * per;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = e / per;
+    dst[r * cols + cols_from + (e - r * per)] = v;
+  }
+}
+
 }  // namespace dsa
 
 using namespace dsa;
@@ -62,11 +75,18 @@ using namespace dsa;
 namespace {
 
 constexpr uint64_t kWaitBudgetNs = 2000000000ull;   // 2 s per bounded wait
+// budget of the indexer's pipeline waits (dsa_set_wait_budget_ns, a test setting)
+std::atomic<uint64_t> g_indexer_wait_ns{kWaitBudgetNs};
 constexpr size_t kAlign = 256;
 constexpr int kPrefillNQ = 4;                       // queries per prefill indexer work item
 constexpr int kMergeThreads = 1024;                  // decode merge: one CTA per sequence
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Prefill items long enough for the indexer's sampled threshold exist (see indexer_topk.cuh).
+bool sampled_threshold(const dsa_dims& d, int32_t topk) {
+  return d.n_q > 1 && topk >= kSpecMinTopk && d.max_len >= kSpecMinTiles * kKeyTile;
+}
 
 bool is_production(const dsa_dims& d) {
   return d.n_idx_heads == kIdxHeads && d.idx_dim == kIdxDim && d.n_heads == kHeads && d.d_latent == kDv &&
@@ -94,7 +114,10 @@ dsa_status check_dims(const dsa_dims* d, int32_t topk) {
 struct Layout {
   size_t status = 0;                     // 256 B: status word + detail
   size_t part_keys = 0, part_pos = 0, part_count = 0;   // decode partial top-k
+  size_t redo_flag = 0, redo_list = 0, redo_count = 0;  // prefill items queued for the exact pass
   size_t idx = 0;                        // forward's selection when out_idx == NULL
+  size_t mask = 0, extent = 0;           // masked dense mode: bitmap rows and extents
+  int32_t mask_words = 0;
   size_t q_idx = 0, w = 0, k_idx = 0, q = 0, kv = 0, out = 0, lse = 0;  // padded copies
   size_t total = 0;
   int32_t n_chunks = 0;
@@ -115,7 +138,18 @@ Layout make_layout(const dsa_dims& d, int32_t topk) {
     L.part_pos = off; off = align_up(off + slots * topk * 4);
     L.part_count = off; off = align_up(off + slots * 4);
   }
+  if (sampled_threshold(d, topk)) {
+    const size_t items = static_cast<size_t>(d.batch) * ((d.n_q + kPrefillNQ - 1) / kPrefillNQ);
+    L.redo_flag = off; off = align_up(off + items * 4);
+    L.redo_list = off; off = align_up(off + items * 4);
+    L.redo_count = off; off = align_up(off + 4);
+  }
   L.idx = off; off = align_up(off + static_cast<size_t>(T) * topk * 4);
+  if (d.max_len <= kMaskMaxLen) {
+    L.mask_words = 2 * ((d.max_len + kBlk - 1) / kBlk);      // two words per 64-row block
+    L.mask = off; off = align_up(off + static_cast<size_t>(T) * L.mask_words * 4);
+    L.extent = off; off = align_up(off + static_cast<size_t>(T) * 4);
+  }
   L.padded = !is_production(d);
   if (L.padded) {
     L.q_idx = off; off = align_up(off + static_cast<size_t>(T) * kIdxHeads * kIdxDim);
@@ -133,6 +167,9 @@ Layout make_layout(const dsa_dims& d, int32_t topk) {
 struct DeviceInfo {
   int sms = 0;
   bool sm100 = false;
+  // the prefill indexer moves registers between warpgroups with setmaxnreg, which is sound only
+  // for the register count its split was computed for
+  bool indexer_regs_ok = false;
 };
 
 DeviceInfo device_info() {
@@ -154,8 +191,14 @@ DeviceInfo device_info() {
                          IdxCfg<kPrefillNQ>::SMEM_BYTES);
     cudaFuncSetAttribute(indexer_topk_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          IdxCfg<1>::SMEM_BYTES);
-    cudaFuncSetAttribute(sparse_mla_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(sparse_mla_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          AttnCfg::SMEM_BYTES);
+    cudaFuncSetAttribute(sparse_mla_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         AttnCfg::SMEM_BYTES);
+    cudaFuncSetAttribute(indexer_kl_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, KlCfg::SMEM_BYTES);
+    cudaFuncAttributes fa{};
+    cache[dev].indexer_regs_ok = cudaFuncGetAttributes(&fa, indexer_topk_kernel<kPrefillNQ>) == cudaSuccess &&
+                                 fa.numRegs == IdxCfg<kPrefillNQ>::LAUNCH_REGS;
     have[dev] = true;
   }
   return cache[dev];
@@ -204,6 +247,20 @@ bool encode_q_bf16(CUtensorMap* map, const void* base, uint64_t rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Latent cache as a 3-D bf16 tensor [1, rows = B*max_len, 576 dims], box {64 dims, box_rows, 1},
+// 128-byte swizzle: one box is one swizzle-atom column of box_rows rows.
+bool encode_kv_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDqk), rows, 1};
+  const cuuint64_t strides[2] = {kDqk * 2, rows * kDqk * 2};
+  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 dsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
@@ -219,6 +276,15 @@ cudaError_t launch_pad(const T* src, T* dst, int64_t rows, int hs, int ds, int h
 }
 
 template <typename T>
+cudaError_t launch_fill(T* dst, int64_t rows, int cols_from, int cols, T v, cudaStream_t st) {
+  const int64_t total = rows * (cols - cols_from);
+  if (total <= 0) return cudaSuccess;
+  const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 65535));
+  fill_cols_kernel<T><<<blocks, 256, 0, st>>>(dst, rows, cols_from, cols, v);
+  return cudaGetLastError();
+}
+
+template <typename T>
 cudaError_t launch_unpad(const T* src, T* dst, int64_t rows, int hs, int ds, int hd, int dd, cudaStream_t st) {
   const int64_t total = rows * hd * dd;
   if (total == 0) return cudaSuccess;
@@ -230,7 +296,7 @@ cudaError_t launch_unpad(const T* src, T* dst, int64_t rows, int hs, int ds, int
 // ----------------------------------------------------------------------------- indexer launch
 dsa_status run_indexer(const dsa_dims& d, const uint8_t* q_idx, const __nv_bfloat16* w, const uint8_t* k_idx,
                        const float* scales, const int32_t* lengths, int32_t topk, int32_t* out_idx,
-                       uint8_t* ws, const Layout& L, cudaStream_t st) {
+                       float* out_scores, uint8_t* ws, const Layout& L, cudaStream_t st) {
   const DeviceInfo dev = device_info();
   IndexerParams p{};
   p.q_idx = q_idx;
@@ -239,12 +305,13 @@ dsa_status run_indexer(const dsa_dims& d, const uint8_t* q_idx, const __nv_bfloa
   p.k_scale = scales + static_cast<size_t>(d.batch) * d.n_q;
   p.lengths = lengths;
   p.out_idx = out_idx;
+  p.out_scores = out_scores;
   p.status = reinterpret_cast<uint32_t*>(ws + L.status);
   p.batch = d.batch;
   p.n_q = d.n_q;
   p.max_len = d.max_len;
   p.topk = topk;
-  p.wait_budget_ns = kWaitBudgetNs;
+  p.wait_budget_ns = g_indexer_wait_ns.load(std::memory_order_relaxed);
   CUtensorMap map_q, map_k;
   if (!encode_rows_u8(&map_k, k_idx, static_cast<uint64_t>(d.max_len), static_cast<uint64_t>(d.batch), kKeyTile))
     return DSA_ERR_CUDA;
@@ -261,24 +328,44 @@ dsa_status run_indexer(const dsa_dims& d, const uint8_t* q_idx, const __nv_bfloa
     indexer_topk_kernel<1><<<grid, IdxCfg<1>::THREADS, IdxCfg<1>::SMEM_BYTES, st>>>(map_q, map_k, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return DSA_ERR_CUDA;
-    MergeParams mp{p.part_keys, p.part_pos, p.part_count, out_idx, L.n_chunks, topk};
+    MergeParams mp{p.part_keys, p.part_pos, p.part_count, out_idx, L.n_chunks, topk, out_scores};
     merge_partials_kernel<kMergeThreads><<<d.batch, kMergeThreads, 0, st>>>(mp);
     return from_cuda(cudaGetLastError());
   }
   p.n_chunks = 0;
   p.n_items = d.batch * ((d.n_q + kPrefillNQ - 1) / kPrefillNQ);
+  if (!dev.indexer_regs_ok) return DSA_ERR_UNSUPPORTED;   // a build whose register count breaks the split
   if (!encode_rows_u8(&map_q, q_idx, static_cast<uint64_t>(d.n_q) * kIdxHeads, static_cast<uint64_t>(d.batch),
                       kPrefillNQ * kIdxHeads))
     return DSA_ERR_CUDA;
+  const bool spec = sampled_threshold(d, topk);
+  if (spec) {
+    // items whose sampled threshold fails are queued during the first launch and rerun exactly
+    // by the second; the queue's length starts at zero
+    p.spec = 1;
+    p.redo_flag = reinterpret_cast<uint32_t*>(ws + L.redo_flag);
+    p.redo_list = reinterpret_cast<int32_t*>(ws + L.redo_list);
+    p.redo_count = reinterpret_cast<uint32_t*>(ws + L.redo_count);
+    if (cudaMemsetAsync(p.redo_count, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
+  }
   const int grid = std::min(p.n_items, dev.sms);
   indexer_topk_kernel<kPrefillNQ><<<grid, IdxCfg<kPrefillNQ>::THREADS, IdxCfg<kPrefillNQ>::SMEM_BYTES, st>>>(map_q,
                                                                                                         map_k, p);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  if (spec) {
+    IndexerParams px = p;
+    px.spec = 0;
+    px.item_list = p.redo_list;
+    px.item_count = p.redo_count;
+    indexer_topk_kernel<kPrefillNQ><<<grid, IdxCfg<kPrefillNQ>::THREADS, IdxCfg<kPrefillNQ>::SMEM_BYTES, st>>>(
+        map_q, map_k, px);
+  }
   return from_cuda(cudaGetLastError());
 }
 
 dsa_status run_attention(const dsa_dims& d, const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
                          int32_t topk, __nv_bfloat16* out, float* lse, uint8_t* ws, const Layout& L,
-                         cudaStream_t st) {
+                         cudaStream_t st, bool masked) {
   const DeviceInfo dev = device_info();
   AttnParams p{};
   p.q = q;
@@ -293,10 +380,25 @@ dsa_status run_attention(const dsa_dims& d, const __nv_bfloat16* q, const __nv_b
   p.n_queries = d.batch * d.n_q;
   p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
   p.wait_budget_ns = kWaitBudgetNs;
-  CUtensorMap map_q;
+  CUtensorMap map_q, map_a, map_b;
   if (!encode_q_bf16(&map_q, q, static_cast<uint64_t>(p.n_queries) * kHeads)) return DSA_ERR_CUDA;
   const int clusters = std::max(1, std::min(p.n_queries, dev.sms / 2));
-  sparse_mla_attn_kernel<<<2 * clusters, AttnCfg::THREADS, AttnCfg::SMEM_BYTES, st>>>(map_q, p);
+  if (!masked) {
+    sparse_mla_attn_kernel<false><<<2 * clusters, AttnCfg::THREADS, AttnCfg::SMEM_BYTES, st>>>(map_q, map_q, map_q, p);
+    return from_cuda(cudaGetLastError());
+  }
+  // masked dense mode: the bitmap of each query's attended positions, then whole 64-row blocks
+  // of its causal prefix by TMA
+  p.mask = reinterpret_cast<const uint32_t*>(ws + L.mask);
+  p.extent = reinterpret_cast<const int32_t*>(ws + L.extent);
+  p.mask_words = L.mask_words;
+  const uint64_t rows = static_cast<uint64_t>(d.batch) * d.max_len;
+  if (!encode_kv_bf16(&map_a, kv, rows, 32) || !encode_kv_bf16(&map_b, kv, rows, kBlk)) return DSA_ERR_CUDA;
+  mask_rows_kernel<<<p.n_queries, 256, 0, st>>>(idx, topk, d.max_len, L.mask_words,
+                                                reinterpret_cast<uint32_t*>(ws + L.mask),
+                                                reinterpret_cast<int32_t*>(ws + L.extent), p.status);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  sparse_mla_attn_kernel<true><<<2 * clusters, AttnCfg::THREADS, AttnCfg::SMEM_BYTES, st>>>(map_q, map_a, map_b, p);
   return from_cuda(cudaGetLastError());
 }
 
@@ -380,9 +482,9 @@ dsa_status dsa_workspace_init(void* ws, size_t ws_bytes, dsa_stream_t stream) {
   return from_cuda(cudaMemsetAsync(ws, 0, kAlign, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-dsa_status dsa_indexer_topk(const dsa_dims* dims, const void* q_idx, const void* w, const void* k_idx,
-                            const float* scales, const int32_t* lengths, int32_t topk, int32_t* out_idx, void* ws,
-                            size_t ws_bytes, dsa_stream_t stream) {
+dsa_status dsa_indexer_topk_scores(const dsa_dims* dims, const void* q_idx, const void* w, const void* k_idx,
+                                   const float* scales, const int32_t* lengths, int32_t topk, int32_t* out_idx,
+                                   float* out_scores, void* ws, size_t ws_bytes, dsa_stream_t stream) {
   dsa_status s = check_dims(dims, topk);
   if (s != DSA_OK) return s;
   const dsa_dims& d = *dims;
@@ -391,19 +493,26 @@ dsa_status dsa_indexer_topk(const dsa_dims* dims, const void* q_idx, const void*
   if (static_cast<int64_t>(d.batch) * d.n_q == 0) return DSA_OK;
   if (!q_idx || !w || !k_idx || !scales || !lengths || !out_idx) return DSA_ERR_INVALID_ARG;
   if (!aligned(q_idx, 16) || !aligned(k_idx, 16) || !aligned(w, 2) || !aligned(scales, 4) ||
-      !aligned(lengths, 4) || !aligned(out_idx, 4))
+      !aligned(lengths, 4) || !aligned(out_idx, 4) || !aligned(out_scores, 4))
     return DSA_ERR_INVALID_ARG;
   if ((s = device_ok()) != DSA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   Prepared pr{};
   if ((s = pad_indexer_inputs(d, q_idx, w, k_idx, wsb, L, st, &pr)) != DSA_OK) return s;
-  return run_indexer(d, pr.q_idx, pr.w, pr.k_idx, scales, lengths, topk, out_idx, wsb, L, st);
+  return run_indexer(d, pr.q_idx, pr.w, pr.k_idx, scales, lengths, topk, out_idx, out_scores, wsb, L, st);
 }
 
-dsa_status dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void* latent_kv, const int32_t* idx,
-                               int32_t topk, void* out, float* lse, void* ws, size_t ws_bytes,
-                               dsa_stream_t stream) {
+dsa_status dsa_indexer_topk(const dsa_dims* dims, const void* q_idx, const void* w, const void* k_idx,
+                            const float* scales, const int32_t* lengths, int32_t topk, int32_t* out_idx, void* ws,
+                            size_t ws_bytes, dsa_stream_t stream) {
+  return dsa_indexer_topk_scores(dims, q_idx, w, k_idx, scales, lengths, topk, out_idx, nullptr, ws, ws_bytes,
+                                 stream);
+}
+
+static dsa_status attention_call(const dsa_dims* dims, const void* q, const void* latent_kv, const int32_t* idx,
+                                 int32_t topk, void* out, float* lse, void* ws, size_t ws_bytes, dsa_stream_t stream,
+                                 bool masked) {
   dsa_status s = check_dims(dims, topk);
   if (s != DSA_OK) return s;
   const dsa_dims& d = *dims;
@@ -413,6 +522,7 @@ dsa_status dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void* 
   if (!q || !latent_kv || !idx || !out || !lse) return DSA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(latent_kv, 16) || !aligned(idx, 4) || !aligned(out, 16) || !aligned(lse, 4))
     return DSA_ERR_INVALID_ARG;
+  if (masked && d.max_len > kMaskMaxLen) return DSA_ERR_UNSUPPORTED;
   if ((s = device_ok()) != DSA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -421,7 +531,7 @@ dsa_status dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void* 
   const int64_t T = static_cast<int64_t>(d.batch) * d.n_q;
   __nv_bfloat16* o = L.padded ? reinterpret_cast<__nv_bfloat16*>(wsb + L.out) : static_cast<__nv_bfloat16*>(out);
   float* ls = L.padded ? reinterpret_cast<float*>(wsb + L.lse) : lse;
-  if ((s = run_attention(d, pr.q, pr.kv, idx, topk, o, ls, wsb, L, st)) != DSA_OK) return s;
+  if ((s = run_attention(d, pr.q, pr.kv, idx, topk, o, ls, wsb, L, st, masked)) != DSA_OK) return s;
   if (L.padded) {
     if (launch_unpad<__nv_bfloat16>(o, static_cast<__nv_bfloat16*>(out), T, kHeads, kDv, d.n_heads, d.d_latent,
                                     st) != cudaSuccess ||
@@ -429,6 +539,65 @@ dsa_status dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void* 
       return DSA_ERR_CUDA;
   }
   return DSA_OK;
+}
+
+dsa_status dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void* latent_kv, const int32_t* idx,
+                               int32_t topk, void* out, float* lse, void* ws, size_t ws_bytes,
+                               dsa_stream_t stream) {
+  return attention_call(dims, q, latent_kv, idx, topk, out, lse, ws, ws_bytes, stream, false);
+}
+
+dsa_status dsa_masked_mqa_attn(const dsa_dims* dims, const void* q, const void* latent_kv, const int32_t* idx,
+                               int32_t topk, void* out, float* lse, void* ws, size_t ws_bytes,
+                               dsa_stream_t stream) {
+  return attention_call(dims, q, latent_kv, idx, topk, out, lse, ws, ws_bytes, stream, true);
+}
+
+dsa_status dsa_indexer_kl_loss(const dsa_dims* dims, const void* q, const void* latent_kv, const int32_t* idx,
+                               const float* idx_scores, const float* lse, int32_t topk, float* loss, void* ws,
+                               size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status s = check_dims(dims, topk);
+  if (s != DSA_OK) return s;
+  const dsa_dims& d = *dims;
+  const Layout L = make_layout(d, topk);
+  if ((s = check_ws(ws, ws_bytes, L)) != DSA_OK) return s;
+  if (static_cast<int64_t>(d.batch) * d.n_q == 0) return DSA_OK;
+  if (!q || !latent_kv || !idx || !idx_scores || !lse || !loss) return DSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(latent_kv, 16) || !aligned(idx, 4) || !aligned(idx_scores, 4) || !aligned(lse, 4) ||
+      !aligned(loss, 4))
+    return DSA_ERR_INVALID_ARG;
+  if ((s = device_ok()) != DSA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  Prepared pr{};
+  if ((s = pad_attention_inputs(d, q, latent_kv, wsb, L, st, &pr)) != DSA_OK) return s;
+  const int64_t T = static_cast<int64_t>(d.batch) * d.n_q;
+  const float* lse_in = lse;
+  if (L.padded) {   // the lse of the padded heads is +inf: their weights exp(z - lse) are 0
+    float* pl = reinterpret_cast<float*>(wsb + L.lse);
+    if (launch_pad<float>(lse, pl, T, 1, d.n_heads, 1, kHeads, d.n_heads, kHeads, st) != cudaSuccess ||
+        launch_fill<float>(pl, T, d.n_heads, kHeads, INFINITY, st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    lse_in = pl;
+  }
+  const DeviceInfo dev = device_info();
+  KlParams p{};
+  p.q = pr.q;
+  p.kv = pr.kv;
+  p.idx = idx;
+  p.scores = idx_scores;
+  p.lse = lse_in;
+  p.loss = loss;
+  p.status = reinterpret_cast<uint32_t*>(wsb + L.status);
+  p.n_q = d.n_q;
+  p.max_len = d.max_len;
+  p.topk = topk;
+  p.n_queries = static_cast<int32_t>(T);
+  p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+  p.wait_budget_ns = kWaitBudgetNs;
+  const int grid = static_cast<int>(std::min<int64_t>(T, dev.sms));
+  indexer_kl_kernel<<<grid, KlCfg::THREADS, KlCfg::SMEM_BYTES, st>>>(p);
+  return from_cuda(cudaGetLastError());
 }
 
 dsa_status dsa_forward(const dsa_dims* dims, const void* q_idx, const void* w, const void* k_idx,
@@ -472,7 +641,12 @@ const char* dsa_status_string(dsa_status status) {
   return "unknown status";
 }
 
-int32_t dsa_version(void) { return 100; }
+int32_t dsa_version(void) { return 200; }
+
+dsa_status dsa_set_wait_budget_ns(uint64_t ns) {
+  g_indexer_wait_ns.store(ns == 0 ? kWaitBudgetNs : ns, std::memory_order_relaxed);
+  return DSA_OK;
+}
 
 }  // extern "C"
 
@@ -562,7 +736,7 @@ extern "C" dsa_status dsa_indexer_topk_decode_noalloc(const dsa_dims* dims, cons
   const int grid = std::min(p.n_items, IdxCfg<1>::CTAS_PER_SM * dev.sms);
   indexer_topk_kernel<1><<<grid, IdxCfg<1>::THREADS, IdxCfg<1>::SMEM_BYTES, st>>>(map_q, map_k, p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-  MergeParams mp{p.part_keys, p.part_pos, p.part_count, out_idx, n_chunks, topk};
+  MergeParams mp{p.part_keys, p.part_pos, p.part_count, out_idx, n_chunks, topk, nullptr};
   merge_partials_kernel<kMergeThreads><<<d.batch, kMergeThreads, 0, st>>>(mp);
   return from_cuda(cudaGetLastError());
 }

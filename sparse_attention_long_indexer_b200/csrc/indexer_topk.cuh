@@ -24,6 +24,16 @@
 //  * prefill items cover a query block's whole causal key range and write the final
 //    indices; decode items (one query per sequence) cover a key chunk and write an exact
 //    partial top-k to the workspace, merged by `merge_partials_kernel`.
+//  * sampled threshold (prefill items of at least kSpecMinTiles key tiles, top-k >= kSpecMinTopk):
+//    the item first visits every kSampleStride-th key tile (a stratified sample of its keys)
+//    and selects the sample's r ~ 1.5 k / kSampleStride best; the r-th score becomes the
+//    admission threshold for the other tiles, which then follow in position order. About 1.5 k
+//    keys of the whole range score at least that, so the candidate buffers rarely need a shrink
+//    afterwards. The threshold is a guess, so the item checks it: if a query ends with fewer
+//    than k candidates, or the sample phase dropped candidates that tied with the k-th for
+//    their position, the item is queued and a second launch reruns the queued items with the
+//    exact streaming threshold. Thresholds in a sampled item never exclude ties (the stream is
+//    not in position order), so the final selection settles ties by position as always.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -37,13 +47,17 @@ constexpr int kIdxHeads = 64;     // H_I (padded)
 constexpr int kIdxDim = 128;      // d_I (padded), one 128-byte row per head / key
 constexpr int kKeyTile = 128;     // keys per MMA tile (M)
 constexpr int kDecodeChunk = 8192;  // keys per decode work item
-constexpr int kSyncTiles = 4;       // key tiles between two capacity checks of a candidate buffer
+constexpr int kSyncTiles = 8;       // key tiles between two capacity checks of a candidate buffer
+constexpr int kSampleStride = 16;   // sampled threshold: the sample is every 16th key tile
+constexpr int kSpecMinTiles = 64;   // ... for items with at least this many key tiles
+constexpr int kSpecMinTopk = 1024;  // ... and at least this top-k (the sample's rank is ~ 3 k / 32)
+constexpr int kSampleLimit = 1024;  // candidate count above which the sample phase shrinks its buffer
 
 template <int NQ>
 struct IdxCfg {
   static constexpr int N = NQ * kIdxHeads;                 // accumulator columns per tile
   static constexpr int NBUF = (NQ == 2) ? 4 : 2;           // TMEM accumulators (NBUF * N <= 512)
-  static constexpr int HALVES = (NQ == 4) ? 2 : 1;         // MMAs per tile (query pairs)
+  static constexpr int HALVES = 1;                         // one MMA of N = NQ * 64 per K step
   // few warps: registers for the head weights and all 64 head columns at once
   static constexpr bool WIDE = NQ <= 2;
   static constexpr int CAND = (NQ == 2) ? 6144 : 3584;     // candidate capacity per query
@@ -53,7 +67,15 @@ struct IdxCfg {
   static constexpr int GROUP_THREADS = 128;                // the threads of one query
   static constexpr int PRODUCER_WARP = EPI_WARPS;
   static constexpr int MMA_WARP = EPI_WARPS + 1;
-  static constexpr int THREADS = (EPI_WARPS + 2) * 32;
+  // prefill: the producer and MMA warps and two idle warps form a fifth warpgroup, which gives
+  // registers to the four epilogue warpgroups with setmaxnreg (launched at LAUNCH_REGS each:
+  // the producer warpgroup drops to AUX_REGS, the epilogue warpgroups rise to EPI_REGS)
+  static constexpr bool REG_SPLIT = NQ == 4;
+  static constexpr int AUX_WARPS = REG_SPLIT ? 4 : 2;
+  static constexpr int THREADS = (EPI_WARPS + AUX_WARPS) * 32;
+  static constexpr int LAUNCH_REGS = 96;                   // 65536 / THREADS rounded down to 8
+  static constexpr int AUX_REGS = 32;
+  static constexpr int EPI_REGS = 112;
   static constexpr int STAGES = (NQ == 4) ? 4 : (NQ == 2) ? 6 : 4;
   // decode (one query per item) runs two CTAs per SM, so that two items' epilogues share an SM
   static constexpr int CTAS_PER_SM = (NQ == 1) ? 2 : 1;
@@ -77,6 +99,11 @@ struct IdxCfg {
   static_assert(CAND - kSyncTiles * kKeyTile >= 2048, "a checked buffer must hold the largest k");
   static_assert(NBUF * HALVES <= 4 && TMEM_COLS <= 512, "accumulators");
   static_assert(THREADS <= 1024 && NQ <= 4, "block shape");
+  // setmaxnreg.inc waits until the registers the block was launched with can serve it, so the
+  // split must fit in THREADS x LAUNCH_REGS (the host checks the compiled count at launch)
+  static_assert(!REG_SPLIT || (THREADS * LAUNCH_REGS <= 65536 &&
+                               EPI_WARPS * 32 * EPI_REGS + AUX_WARPS * 32 * AUX_REGS <= THREADS * LAUNCH_REGS),
+                "register split");
   static_assert(Q_BYTES % 1024 == 0 && K_BYTES % 1024 == 0, "swizzle atoms");
 };
 
@@ -87,6 +114,7 @@ struct IndexerParams {
   const float* k_scale;     // [B*max_len]
   const int32_t* lengths;   // [B]
   int32_t* out_idx;         // prefill: [B, n_q, topk]
+  float* out_scores;        // optional, prefill: [B, n_q, topk] index score of each selected position
   uint32_t* part_keys;      // decode: [B, n_chunks, topk]
   int32_t* part_pos;        // decode: [B, n_chunks, topk]
   int32_t* part_count;      // decode: [B, n_chunks]
@@ -94,6 +122,14 @@ struct IndexerParams {
   int32_t batch, n_q, max_len, topk, n_chunks;
   int32_t n_items;
   uint64_t wait_budget_ns;
+  // sampled threshold (prefill): spec enables it; items whose guess fails are queued here
+  int32_t spec;
+  uint32_t* redo_flag;          // [n_items] 1 once the item is queued
+  int32_t* redo_list;           // [n_items] queued items
+  uint32_t* redo_count;         // entries in redo_list (zeroed by the host before the launch)
+  // exact pass over queued items: item j of this launch is item_list[j], j < *item_count
+  const int32_t* item_list;
+  const uint32_t* item_count;
 };
 
 // Bounded wait that ignores the abort flag: used at teardown to let in-flight copies and
@@ -105,10 +141,27 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-// Work item u -> (sequence, first query, key start, key end (exclusive), #tiles).
+// Work item u -> (sequence, first query, key start, key end (exclusive), #tiles, sample tiles).
 struct Item {
-  int32_t b, i0, s_begin, s_end, ntiles, len;
+  int32_t b, i0, s_begin, s_end, ntiles, len, n_s;
 };
+
+// Key tile visited at step t of an item: with a sample phase (n_s > 0) steps 0..n_s-1 visit
+// tiles 0, 16, 32, ... and the later steps the other tiles in increasing order.
+__device__ __forceinline__ int32_t tile_at(const Item& it, int32_t t) {
+  if (it.n_s == 0) return t;
+  if (t < it.n_s) return t * kSampleStride;
+  const int32_t j = t - it.n_s;
+  return j + j / (kSampleStride - 1) + 1;
+}
+
+// The sample's rank r: about 1.5 k scaled to the sampled fraction of the tiles.
+__device__ __forceinline__ uint32_t sample_rank(int32_t topk, const Item& it) {
+  return static_cast<uint32_t>((3 * topk * it.n_s + 2 * it.ntiles - 1) / (2 * it.ntiles));
+}
+
+// Item index of round `round` of this CTA, false when the CTA has no more items.
+__device__ __forceinline__ bool item_at(const IndexerParams& p, int32_t round, int32_t cta, int32_t G, int32_t& u);
 
 template <int NQ>
 __device__ __forceinline__ Item make_item(const IndexerParams& p, int32_t u) {
@@ -138,12 +191,26 @@ __device__ __forceinline__ Item make_item(const IndexerParams& p, int32_t u) {
   }
   const int32_t span = it.s_end - it.s_begin;
   it.ntiles = span > 0 ? (span + kKeyTile - 1) / kKeyTile : 0;
+  it.n_s = (NQ > 1 && p.spec && it.ntiles >= kSpecMinTiles && p.topk >= kSpecMinTopk)
+               ? (it.ntiles + kSampleStride - 1) / kSampleStride
+               : 0;
   return it;
 }
 
 // Item sequence of CTA `cta` among `G`: snake order over rounds.
 __device__ __forceinline__ int32_t item_of(int32_t round, int32_t cta, int32_t G) {
   return round * G + ((round & 1) ? (G - 1 - cta) : cta);
+}
+
+__device__ __forceinline__ bool item_at(const IndexerParams& p, int32_t round, int32_t cta, int32_t G, int32_t& u) {
+  const int32_t j = item_of(round, cta, G);
+  if (p.item_list == nullptr) {
+    u = j;
+    return j < p.n_items;
+  }
+  if (j >= static_cast<int32_t>(__ldg(p.item_count))) return false;
+  u = __ldg(p.item_list + j);
+  return true;
 }
 
 template <int NQ>
@@ -196,15 +263,16 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
   }
   const int32_t G = gridDim.x;
   const int32_t cta = blockIdx.x;
-  if (NQ == 1) {
-    // decode: slot u of the partial lists belongs to work item u, which only this CTA runs.
-    // Its count starts at zero here, before the barrier, so a slot this CTA never reaches
-    // (after an aborted wait) reads as empty in the merge instead of holding an earlier
-    // call's count.
+  if (NQ == 1 || (p.spec && p.item_list == nullptr)) {
+    // Per-item words that only this CTA writes start at zero here, before the barrier. Decode:
+    // slot u of the partial lists belongs to item u, so a slot this CTA never reaches (after an
+    // aborted wait) reads as empty in the merge instead of holding an earlier call's count.
+    // Sampled prefill: item u's queued flag.
     for (int32_t r = static_cast<int32_t>(threadIdx.x);; r += static_cast<int32_t>(blockDim.x)) {
       const int32_t u = item_of(r, cta, G);
       if (u >= p.n_items) break;
-      p.part_count[u] = 0;
+      if (NQ == 1) p.part_count[u] = 0;
+      else p.redo_flag[u] = 0u;
     }
   }
   tc_fence_before();
@@ -213,6 +281,10 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
   const uint32_t tmem = *tmem_slot;
   Waiter wt{p.status, abort_flag, p.wait_budget_ns, 1u};
 
+  if (warp >= static_cast<uint32_t>(C::EPI_WARPS)) {
+    // producer, MMA issuer and (prefill) two idle warps: one warpgroup, which hands registers
+    // to the epilogue warpgroups
+    if constexpr (C::REG_SPLIT) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::AUX_REGS));
   if (warp == C::PRODUCER_WARP) {
     // ------------------------------------------------------------- TMA producer
     if (lane == 0) {
@@ -221,8 +293,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       uint32_t stage = 0, phase = 0, qph = 0;
       uint32_t used = 0, last_par = 0, q_out = 0;  // per stage: issued at least once / parity of last issue
       for (int32_t r = 0;; ++r) {
-        const int32_t u = item_of(r, cta, G);
-        if (u >= p.n_items || wt.aborted()) break;
+        int32_t u;
+        if (!item_at(p, r, cta, G, u) || wt.aborted()) break;
         const Item it = make_item<NQ>(p, u);
         if (it.ntiles == 0) continue;
         if (!wt.wait(q_empty, qph ^ 1u, 1)) break;
@@ -235,7 +307,7 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
           if (!wt.wait(k_empty(stage), phase ^ 1u, 2)) { ok = false; break; }
           mbar_expect_tx(k_full(stage), C::K_BYTES);
           tma_load_3d(sbase + C::OFF_K + stage * C::K_BYTES, &map_k, k_full(stage), 0,
-                      it.s_begin + t * kKeyTile, it.b);
+                      it.s_begin + tile_at(it, t) * kKeyTile, it.b);
           used |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -245,8 +317,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       // drain: every issued copy must have landed before the CTA may exit. Waiting on a
       // completed phase returns at once; after an abort this bounds the in-flight copies.
       for (int s = 0; s < C::STAGES; ++s)
-        if (used & (1u << s)) drain_wait(k_full(s), (last_par >> s) & 1u, p.wait_budget_ns);
-      if (q_out & 1u) drain_wait(q_full, (q_out >> 1) & 1u, p.wait_budget_ns);
+        if (used & (1u << s)) drain_wait(k_full(s), (last_par >> s) & 1u, kDrainBudgetNs);
+      if (q_out & 1u) drain_wait(q_full, (q_out >> 1) & 1u, kDrainBudgetNs);
     }
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------- MMA issuer
@@ -254,8 +326,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       constexpr uint32_t idesc = make_idesc(0, 0, 0, 0, kKeyTile, C::NH);
       uint32_t stage = 0, phase = 0, qph = 0, g = 0;
       for (int32_t r = 0;; ++r) {
-        const int32_t u = item_of(r, cta, G);
-        if (u >= p.n_items || wt.aborted()) break;
+        int32_t u;
+        if (!item_at(p, r, cta, G, u) || wt.aborted()) break;
         const Item it = make_item<NQ>(p, u);
         if (it.ntiles == 0) continue;
         if (!wt.wait(q_full, qph, 4)) break;
@@ -289,9 +361,11 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       }
       // drain: all MMAs complete before TMEM is released
       tc_commit(mma_done);
-      drain_wait(mma_done, 0, p.wait_budget_ns);
+      drain_wait(mma_done, 0, kDrainBudgetNs);
     }
+  }
   } else {
+    if constexpr (C::REG_SPLIT) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::EPI_REGS));
     // ------------------------------------------------------------- epilogue warps
     // Warps 4q .. 4q+3 own query q of the block, one TMEM lane quarter (32 keys) each; the
     // four run as a group with their own named barrier (1 + q), candidate buffer and select
@@ -320,8 +394,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     };
     bool stop = false;
     for (int32_t r = 0; !stop; ++r) {
-      const int32_t u = item_of(r, cta, G);
-      if (u >= p.n_items) break;
+      int32_t u;
+      if (!item_at(p, r, cta, G, u)) break;
       const Item it = make_item<NQ>(p, u);
       const int32_t i = it.i0 + static_cast<int32_t>(q);
       const bool q_valid = NQ == 1 || i < p.n_q;
@@ -352,23 +426,22 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       }
       const float* ks_row = p.k_scale + static_cast<size_t>(it.b) * p.max_len;
       const int32_t s_lane = it.s_begin + static_cast<int32_t>(quarter * 32 + lane);
-      // the key scale of the next tile is loaded one tile ahead (clamped address; the value
-      // of a key past the range is never used)
-      auto key_scale = [&](int32_t t) -> float {
-        return __ldg(ks_row + min(s_lane + t * kKeyTile, it.s_end - 1));
-      };
-      float ks_next = key_scale(0);
-      // Candidates are appended at the capacity checks, not per tile: bit j of pbits says that
-      // this lane's key of the tile j tiles back passed, pk[j] is its score key. A check thus
-      // takes one atomic per warp for up to kSyncTiles tiles.
-      uint32_t pk[kSyncTiles];
-      uint32_t pbits = 0;
+      // this lane's key at step t; the next step's key and its scale are fetched one step ahead
+      // (clamped address: the scale of a key past the range is never used)
+      auto key_at = [&](int32_t t) -> int32_t { return s_lane + tile_at(it, t) * kKeyTile; };
+      int32_t s_next = key_at(0);
+      float ks_next = __ldg(ks_row + min(s_next, it.s_end - 1));
+      // a sampled item may drop candidates that tie with the sample's selection for their
+      // position; its queries are then rerun exactly
+      bool sample_tie = false;
+      const uint32_t lanes_below = (1u << lane) - 1u;
       for (int32_t t = 0; t < it.ntiles; ++t, ++g) {
         const uint32_t buf = g % C::NBUF, acc_ph = (g / C::NBUF) & 1u;
-        const int32_t s = s_lane + t * kKeyTile;
-        const bool in_range = s < it.s_end;
+        const int32_t s = s_next;
         const float ks = ks_next;
-        ks_next = key_scale(t + 1);
+        s_next = key_at(t + 1);
+        ks_next = __ldg(ks_row + min(s_next, it.s_end - 1));
+        const bool in_range = s < it.s_end;
         // every lane waits (no divergent branch); the warp then runs the collective TMEM loads
         const bool ok = __all_sync(0xffffffffu, wt.wait(acc_full(buf, half), acc_ph, 8)) != 0;
         bool pass = false;
@@ -427,54 +500,48 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
           const bool valid = in_range && s <= qpos;
           pass = valid && (key > thr_r || (key == thr_r && strict_r == 0));
         }
-#pragma unroll
-        for (int j = kSyncTiles - 1; j > 0; --j) pk[j] = pk[j - 1];
-        pk[0] = key;
-        pbits = (pbits << 1) | (pass ? 1u : 0u);
-        // capacity check every kSyncTiles tiles: between two checks at most kSyncTiles * 128
-        // candidates arrive, and a check leaves at most CAND - kSyncTiles * 128
-        if (t % kSyncTiles != kSyncTiles - 1 && t + 1 != it.ntiles) continue;
-        {
-          // append this warp's passes of the tiles since the last check (tile t - j for bit j)
-          const uint32_t lt = (1u << lane) - 1u;
-          uint32_t off[kSyncTiles];
-          uint32_t total = 0;
-#pragma unroll
-          for (int j = 0; j < kSyncTiles; ++j) {
-            const uint32_t mj = __ballot_sync(0xffffffffu, (pbits >> j) & 1u);
-            off[j] = total + __popc(mj & lt);
-            total += __popc(mj);
+        // this tile's passes go into the buffer at once: one ballot, and one atomic for a warp
+        // with any pass (after the first few tiles most warps have none)
+        const uint32_t passed = __ballot_sync(0xffffffffu, pass);
+        if (passed != 0u) {
+          uint32_t base = 0;
+          if (lane == 0) base = atomicAdd(&q_count[q], static_cast<uint32_t>(__popc(passed)));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (pass) {
+            const uint32_t at = base + static_cast<uint32_t>(__popc(passed & lanes_below));
+            cq_keys[at] = key;
+            cq_pos[at] = s;
           }
-          if (total) {
-            uint32_t base = 0;
-            if (lane == 0) base = atomicAdd(&q_count[q], total);
-            base = __shfl_sync(0xffffffffu, base, 0);
-#pragma unroll
-            for (int j = 0; j < kSyncTiles; ++j) {
-              if ((pbits >> j) & 1u) {
-                cq_keys[base + off[j]] = pk[j];
-                cq_pos[base + off[j]] = s - j * kKeyTile;
-              }
-            }
-          }
-          pbits = 0;
         }
+        // capacity check every kSyncTiles tiles: between two checks at most kSyncTiles * 128
+        // candidates arrive, and a check leaves at most CAND - kSyncTiles * 128 (also at the
+        // end of a sample phase)
+        const bool boundary = t + 1 == it.n_s;
+        if (t % kSyncTiles != kSyncTiles - 1 && t + 1 != it.ntiles && !boundary) continue;
         if (uniform_stop()) { stop = true; break; }
-        const uint32_t n = q_count[q];
-        if (n > static_cast<uint32_t>(C::CAND - kSyncTiles * kKeyTile)) {
+        uint32_t n = q_count[q];
+        // the sample phase selects the sample's r best, under a lower capacity limit
+        const bool sampling = t < it.n_s;
+        const uint32_t tgt = sampling ? sample_rank(p.topk, it) : static_cast<uint32_t>(p.topk);
+        const uint32_t limit = sampling ? static_cast<uint32_t>(kSampleLimit)
+                                        : static_cast<uint32_t>(C::CAND - kSyncTiles * kKeyTile);
+        if (n > limit) {
           // cheap range-histogram shrink; the exact select only if it frees too little
           uint32_t thr = 0;
-          const uint32_t m = shrink_candidates<C::GROUP_THREADS, C::MAXPER>(
-              cq_keys, cq_pos, n, static_cast<uint32_t>(p.topk), gsel, gtid, bar_id, &thr);
+          const uint32_t m = shrink_candidates<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, n, tgt, gsel, gtid,
+                                                                            bar_id, &thr);
           // the exact select when the shrink freed less than half of the usable space
-          if (m > static_cast<uint32_t>(C::CAND - kSyncTiles * kKeyTile + p.topk) / 2) {
-            const uint32_t vk = select_exact<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, m,
-                                                                          static_cast<uint32_t>(p.topk), gsel, gtid,
-                                                                          bar_id);
+          if (m > (limit + tgt) / 2) {
+            bool tied = false;
+            const uint32_t vk =
+                select_exact<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, m, tgt, gsel, gtid, bar_id, &tied);
+            if (sampling && tied) sample_tie = true;
             if (gtid == 0) {
-              q_count[q] = p.topk;
+              q_count[q] = tgt;
               q_thr[q] = vk;
-              q_strict[q] = 1;
+              // a strict threshold relies on later keys having larger positions: only in
+              // position order
+              q_strict[q] = it.n_s == 0 ? 1u : 0u;
             }
           } else if (gtid == 0) {
             q_count[q] = m;
@@ -484,12 +551,33 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
           named_barrier(bar_id, C::GROUP_THREADS);
           thr_r = q_thr[q];
           strict_r = q_strict[q];
+          n = q_count[q];
+        }
+        if (boundary && n > tgt) {
+          // end of the sample phase: the sample's r-th best key becomes the admission threshold
+          // (non-strict); every candidate at or above it stays
+          uint32_t kept = 0;
+          const uint32_t v =
+              select_keep_ge<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, n, tgt, gsel, gtid, bar_id, &kept);
+          if (gtid == 0) {
+            q_count[q] = kept;
+            q_thr[q] = max(v, thr_r);
+            q_strict[q] = 0;
+          }
+          named_barrier(bar_id, C::GROUP_THREADS);
+          thr_r = q_thr[q];
+          strict_r = 0;
         }
       }
       if (stop) break;
       // ---- finish the query: exact k, then write
       if (q_valid) {
         uint32_t n = q_count[q];
+        // a sampled item whose threshold kept fewer than k candidates, or dropped ties in its
+        // sample phase, is queued for the exact pass (which rewrites all its queries)
+        if (it.n_s > 0 && (n < static_cast<uint32_t>(p.topk) || sample_tie) && gtid == 0) {
+          if (atomicExch(p.redo_flag + u, 1u) == 0u) p.redo_list[atomicAdd(p.redo_count, 1u)] = u;
+        }
         if (n > static_cast<uint32_t>(p.topk)) {
           select_exact<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, n, static_cast<uint32_t>(p.topk), gsel, gtid,
                                                     bar_id);
@@ -503,9 +591,15 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
           }
           if (gtid == 0) p.part_count[slot] = static_cast<int32_t>(n);
         } else {
-          int32_t* dst = p.out_idx + (static_cast<size_t>(it.b) * p.n_q + i) * p.topk;
+          const size_t row = (static_cast<size_t>(it.b) * p.n_q + i) * p.topk;
+          int32_t* dst = p.out_idx + row;
           for (uint32_t j = gtid; j < static_cast<uint32_t>(p.topk); j += C::GROUP_THREADS)
             dst[j] = j < n ? cq_pos[j] : -1;
+          if (p.out_scores != nullptr) {
+            float* sdst = p.out_scores + row;
+            for (uint32_t j = gtid; j < static_cast<uint32_t>(p.topk); j += C::GROUP_THREADS)
+              sdst[j] = j < n ? key_score(cq_keys[j]) : -INFINITY;
+          }
         }
       }
       named_barrier(bar_id, C::GROUP_THREADS);
@@ -529,6 +623,7 @@ struct MergeParams {
   const int32_t* part_count;
   int32_t* out_idx;        // [B, n_q(=1), topk]
   int32_t n_chunks, topk;
+  float* out_scores;       // optional [B, n_q(=1), topk]
 };
 
 template <int T>
@@ -646,10 +741,16 @@ __global__ void __launch_bounds__(T) merge_partials_kernel(const MergeParams p) 
     if (lane == 0 && m) base = atomicAdd(&sc.out_count, __popc(m));
     base = __shfl_sync(0xffffffffu, base, 0);
     const uint32_t at = base + __popc(m & ((1u << lane) - 1u));
-    if (keep && at < k) dst[at] = ps;
+    if (keep && at < k) {
+      dst[at] = ps;
+      if (p.out_scores != nullptr) p.out_scores[static_cast<size_t>(b) * p.topk + at] = key_score(key);
+    }
   });
   __syncthreads();
-  for (uint32_t j = min(sc.out_count, k) + tid; j < k; j += T) dst[j] = -1;
+  for (uint32_t j = min(sc.out_count, k) + tid; j < k; j += T) {
+    dst[j] = -1;
+    if (p.out_scores != nullptr) p.out_scores[static_cast<size_t>(b) * p.topk + j] = -INFINITY;
+  }
 }
 
 }  // namespace dsa

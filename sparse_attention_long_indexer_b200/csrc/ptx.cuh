@@ -59,6 +59,11 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
+// `count` arrivals at once on a barrier of another CTA of the cluster, release at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster_n(uint32_t remote_bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(remote_bar), "r"(count)
+               : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -89,8 +94,13 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
   return ok != 0;
 }
 
+// Budget of the teardown drains (in-flight copies and MMAs land before shared memory and TMEM
+// are released). It does not follow the pipeline waits' budget, which a test may shorten.
+constexpr uint64_t kDrainBudgetNs = 2000000000ull;
+
 // Bounded waiting. `abort` is a CTA-shared flag: once any thread times out, every later
-// wait in the CTA returns false immediately, so all roles drain to the kernel's exit.
+// wait in the CTA returns false immediately, so all roles drain to the kernel's exit. A budget
+// under 1 us (a test's setting) is checked on every retry instead of every 64th.
 struct Waiter {
   uint32_t* status;        // global status word (may be null)
   volatile int* abort;     // shared-memory abort flag
@@ -106,7 +116,7 @@ struct Waiter {
     uint32_t spins = 0;
     while (true) {
       if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
-      if ((++spins & 63u) == 0) {
+      if ((++spins & 63u) == 0 || budget_ns < 1000u) {
         if (*abort) return false;
         if (global_timer_ns() - t0 > budget_ns) {
           record_error(status, DSA_ERR_DEVICE_TIMEOUT, (where << 16) | tag);

@@ -18,6 +18,11 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Inverse of score_key: the fp32 score a key was made from.
+__device__ __forceinline__ float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 struct SelectScratch {
   uint32_t hist[256];
   uint32_t bin;     // chosen digit
@@ -212,46 +217,57 @@ __device__ __forceinline__ void compact_candidates(uint32_t* keys, int32_t* pos,
   named_barrier(bar_id, T);
 }
 
-// Keeps exactly k of the n candidates (n > k): the k largest keys, equal keys ranked by the
-// lower position. Returns a threshold key t such that any later candidate with a key <= t
-// (and, being later, a larger position) cannot enter the top k.
+// Key passes over the items held in registers: narrows an adaptive range down to the bin that
+// holds the k-th largest key. Returns the bin's lower edge and `rem`, the places left for the
+// items at or above it once the items above the bin are counted; `ties` says that the bin is a
+// single key value holding more items than places.
+struct KthKey {
+  uint32_t value;
+  uint32_t rem;
+  bool ties;
+};
+
 template <int T, int MAXPER>
-__device__ uint32_t select_exact(uint32_t* keys, int32_t* pos, uint32_t n, uint32_t k, SelectScratch* sc,
-                                 uint32_t tid, uint32_t bar_id) {
-  uint32_t rk[MAXPER];
-  int32_t rp[MAXPER];
-  load_candidates<T, MAXPER>(keys, pos, n, tid, rk, rp);
-  if (tid == 0) sc->out_count = 0;
+__device__ __forceinline__ KthKey kth_key(const uint32_t (&rk)[MAXPER], const int32_t (&rp)[MAXPER], uint32_t k,
+                                          SelectScratch* sc, uint32_t tid, uint32_t bar_id) {
   uint32_t lo, hi;
   group_minmax<T, MAXPER>([&](int j) { return rp[j] >= 0; }, [&](int j) { return rk[j]; }, sc, tid, bar_id, lo, hi);
-  // ---- key passes: narrow the active range to the bin holding the k-th largest key
   uint32_t rem = k, shift = bin_shift(hi - lo), a_lo = lo, a_hi = hi;
-  uint32_t thr = 0, vk = 0;
-  bool ties = false;
   while (true) {
     uint32_t bin, above, cnt;
     hist_pass<true, T, MAXPER>([&](int j) { return rp[j] >= 0 && rk[j] >= a_lo && rk[j] <= a_hi; },
                                [&](int j) { return (rk[j] - a_lo) >> shift; }, rem, sc, tid, bar_id, bin, above, cnt);
     rem -= above;
     const uint32_t blo = a_lo + (bin << shift);
-    if (cnt == rem) {                 // the whole bin is in: keys >= blo are exactly the k
-      thr = blo;
-      break;
-    }
-    if (shift == 0) {                 // a single key value, more items than places: ties
-      vk = blo;
-      ties = true;
-      break;
-    }
+    if (cnt == rem) return KthKey{blo, rem, false};   // the whole bin is in: keys >= blo are exactly k
+    if (shift == 0) return KthKey{blo, rem, true};    // one key value, more items than places
     a_hi = bin_end(blo, shift, a_hi);
     a_lo = blo;
     shift = shift > 8u ? shift - 8u : 0u;
   }
-  if (!ties) {
+}
+
+// Keeps exactly k of the n candidates (n > k): the k largest keys, equal keys ranked by the
+// lower position. Returns a threshold key t such that any later candidate with a key <= t
+// (and, being later, a larger position) cannot enter the top k. `*tied` (if given) is set when
+// candidates equal to the k-th key were dropped for their position.
+template <int T, int MAXPER>
+__device__ uint32_t select_exact(uint32_t* keys, int32_t* pos, uint32_t n, uint32_t k, SelectScratch* sc,
+                                 uint32_t tid, uint32_t bar_id, bool* tied = nullptr) {
+  uint32_t rk[MAXPER];
+  int32_t rp[MAXPER];
+  load_candidates<T, MAXPER>(keys, pos, n, tid, rk, rp);
+  if (tid == 0) sc->out_count = 0;
+  const KthKey kth = kth_key<T, MAXPER>(rk, rp, k, sc, tid, bar_id);
+  if (tied != nullptr) *tied = kth.ties;
+  if (!kth.ties) {
+    const uint32_t thr = kth.value;
     compact_candidates<T, MAXPER>(keys, pos, rk, rp, [&](uint32_t key, int32_t) { return key >= thr; }, sc, bar_id);
     return thr;
   }
   // ---- position passes among the items equal to vk: keep the rem lowest positions
+  const uint32_t vk = kth.value;
+  uint32_t rem = kth.rem;
   uint32_t plo, phi;
   group_minmax<T, MAXPER>([&](int j) { return rp[j] >= 0 && rk[j] == vk; },
                           [&](int j) { return static_cast<uint32_t>(rp[j]); }, sc, tid, bar_id, plo, phi);
@@ -280,6 +296,22 @@ __device__ uint32_t select_exact(uint32_t* keys, int32_t* pos, uint32_t n, uint3
       [&](uint32_t key, int32_t ps) { return key > vk || (key == vk && static_cast<uint32_t>(ps) <= plim); }, sc,
       bar_id);
   return vk;
+}
+
+// Keeps every candidate whose key is at least the k-th largest key value v (ties at v all
+// stay, so k or more remain) and returns v, or the lower edge of a bin that holds exactly the
+// k largest keys. `*kept` receives the number of candidates kept.
+template <int T, int MAXPER>
+__device__ uint32_t select_keep_ge(uint32_t* keys, int32_t* pos, uint32_t n, uint32_t k, SelectScratch* sc,
+                                   uint32_t tid, uint32_t bar_id, uint32_t* kept) {
+  uint32_t rk[MAXPER];
+  int32_t rp[MAXPER];
+  load_candidates<T, MAXPER>(keys, pos, n, tid, rk, rp);
+  if (tid == 0) sc->out_count = 0;
+  const uint32_t v = kth_key<T, MAXPER>(rk, rp, k, sc, tid, bar_id).value;
+  compact_candidates<T, MAXPER>(keys, pos, rk, rp, [&](uint32_t key, int32_t) { return key >= v; }, sc, bar_id);
+  *kept = sc->out_count;
+  return v;
 }
 
 // Cheap shrink used while streaming: one histogram pass over the candidates' key range

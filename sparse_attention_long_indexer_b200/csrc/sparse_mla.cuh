@@ -91,7 +91,7 @@ struct AttnCfg {
   static constexpr int OFF_SCAN = OFF_XMAX + 2 * 128 * 8;
   static constexpr int OFF_INFO = OFF_SCAN + 64;
   static constexpr int OFF_BAR = OFF_INFO + 16;
-  static constexpr int NUM_BARS = 40;
+  static constexpr int NUM_BARS = 45;                    // 40..44: masked-mode copy barriers
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(OFF_VR % 1024 == 0 && OFF_QS % 1024 == 0 && OFF_P % 1024 == 0, "swizzle atoms");
@@ -99,7 +99,13 @@ struct AttnCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(P_BUFS == 1 || P_BUFS == 2, "P buffers");
   static_assert(SB_STAGES <= 4 && VR_STAGES <= 4 && S_BUFS <= 3, "barrier slots");
+  static_assert(SB_STAGES <= 3 && VR_STAGES <= 2, "masked-mode copy barriers");
 };
+
+// Masked dense mode: the longest key range whose attended positions fit the bitmap (see
+// mask_rows_kernel) and the words of a bitmap row.
+constexpr int kMaskMaxLen = 16384;
+constexpr int kMaskMaxWords = kMaskMaxLen / 32;
 
 struct AttnParams {
   const __nv_bfloat16* q;      // [B*n_q, 128, 576]
@@ -111,7 +117,44 @@ struct AttnParams {
   int32_t n_q, max_len, topk, n_queries;
   float scale_log2;            // tau * log2(e)
   uint64_t wait_budget_ns;
+  // masked dense mode: attended positions as a bitmap per query, and one past the last of them
+  const uint32_t* mask;        // [B*n_q, mask_words]
+  const int32_t* extent;       // [B*n_q]
+  int32_t mask_words;
 };
+
+// Masked dense mode, first step: the attended positions of each query as a bitmap of `words`
+// words (bit s%32 of word s/32), and one past the last of them. One CTA per query. Entries < 0
+// are padding; entries >= max_len are reported (DSA_ERR_INDEX_RANGE) and ignored; a position
+// listed twice is attended once.
+__global__ void __launch_bounds__(256) mask_rows_kernel(const int32_t* __restrict__ idx, int32_t topk,
+                                                        int32_t max_len, int32_t words, uint32_t* __restrict__ mask,
+                                                        int32_t* __restrict__ extent, uint32_t* status) {
+  __shared__ uint32_t bm[kMaskMaxWords];
+  __shared__ int32_t last;
+  const int32_t qi = blockIdx.x;
+  for (int32_t w = threadIdx.x; w < words; w += blockDim.x) bm[w] = 0u;
+  if (threadIdx.x == 0) last = -1;
+  __syncthreads();
+  const int32_t* row = idx + static_cast<size_t>(qi) * topk;
+  int32_t mx = -1;
+  for (int32_t j = threadIdx.x; j < topk; j += blockDim.x) {
+    const int32_t v = __ldg(row + j);
+    if (v >= max_len) {
+      record_error(status, DSA_ERR_INDEX_RANGE, static_cast<uint32_t>(qi));
+    } else if (v >= 0) {
+      atomicOr(&bm[v >> 5], 1u << (v & 31));
+      mx = max(mx, v);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(&last, mx);
+  __syncthreads();
+  uint32_t* out = mask + static_cast<size_t>(qi) * words;
+  for (int32_t w = threadIdx.x; w < words; w += blockDim.x) out[w] = bm[w];
+  if (threadIdx.x == 0) extent[qi] = last + 1;
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -143,8 +186,14 @@ __device__ __forceinline__ void commit2(uint32_t bar_cluster_addr) {
                : "memory");
 }
 
+// kDense: the masked dense mode. Block b of a query is then its positions 64b .. 64b+63, loaded
+// whole by TMA tile copies (map_kv_a: boxes of 32 rows, map_kv_b: boxes of 64 rows, both over the
+// latent cache as [B * max_len rows, 576 dims]), and the softmax masks the positions that are not
+// in the query's bitmap; blocks run up to the query's extent (one past its last attended position).
+template <bool kDense>
 __global__ void __launch_bounds__(AttnCfg::THREADS, 1) __cluster_dims__(2, 1, 1)
-sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnParams p) {
+sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv_a,
+                       const __grid_constant__ CUtensorMap map_kv_b, const AttnParams p) {
   using C = AttnCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -180,6 +229,9 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
   auto p_local = [&](uint32_t j) { return j ? B(11) : B(30); };   // odd CTA: its softmax warps
   const uint32_t o_empty2 = B(28);
   const uint32_t mma_done = B(29);
+  // masked dense mode: a stage's TMA copies landed in this CTA (local, one expect_tx arrive)
+  auto sb_tma = [&](uint32_t s) { return B(40 + static_cast<int>(s)); };
+  auto vr_tma = [&](uint32_t s) { return B(43 + static_cast<int>(s)); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -216,6 +268,8 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
     }
     mbar_init(o_empty2, 2 * C::SOFTMAX_WARPS);
     mbar_init(mma_done, 2);
+    for (uint32_t i = 0; i < 3u; ++i) mbar_init(sb_tma(i), 1);
+    for (uint32_t i = 0; i < 2u; ++i) mbar_init(vr_tma(i), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -277,10 +331,14 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         // and >= max_len (reported) are masked wherever they appear: their rows are gathered as
         // zeros and their logits set to -inf, so blocks are read straight from the index row.
         int32_t last = -1;
-        for (int32_t j = static_cast<int32_t>(gtid); j < p.topk; j += C::GROUP_THREADS) {
-          const int32_t v = __ldg(idx_row + j);
-          if (v >= p.max_len) record_error(p.status, DSA_ERR_INDEX_RANGE, static_cast<uint32_t>(qi));
-          if (v >= 0 && v < p.max_len) last = j;
+        if constexpr (kDense) {
+          last = __ldg(p.extent + qi) - 1;                // blocks cover positions 0 .. extent-1
+        } else {
+          for (int32_t j = static_cast<int32_t>(gtid); j < p.topk; j += C::GROUP_THREADS) {
+            const int32_t v = __ldg(idx_row + j);
+            if (v >= p.max_len) record_error(p.status, DSA_ERR_INDEX_RANGE, static_cast<uint32_t>(qi));
+            if (v >= 0 && v < p.max_len) last = j;
+          }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
@@ -333,86 +391,141 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
           ok = false;
         }
         ++qq;
-        // ---- the ring of this group. Thread (r0, cc) copies 16-byte chunk cc of every 128-byte
-        // segment of block rows r0, r0 + GROUP_THREADS/8, ...: the row indices are read once per block and each
-        // copy is a constant offset from the row's base, so copies issue back to back.
-        const __nv_bfloat16* kv_seq = p.kv + static_cast<size_t>(qi / p.n_q) * p.max_len * kDqk;
-        const uint32_t cc = gtid & 7u, r0 = gtid >> 3;
-        const int32_t own0 = 32 * static_cast<int32_t>(rank);
-        const uint32_t seg0 = 128u * rank;               // group B: segments 2r, 2r+1, 4+2r, 5+2r
-        // block row r of block b: its row of the latent cache, or -1 when masked (padding, past the
-        // extent, or out of range); read from the index row one block ahead of its gathers
-        constexpr int RS = C::GROUP_THREADS / 8;       // rows per pass
-        constexpr int NRA = 32 / RS, NRB = kBlk / RS;  // rows per thread: logits ring, output ring
-        auto row_of = [&](int32_t b, int32_t r) -> int32_t {
-          const int32_t j = b * kBlk + r;
-          const int32_t v = j < total ? __ldg(idx_row + j) : -1;
-          return (v >= 0 && v < p.max_len) ? v : -1;
-        };
-        int32_t rows_a[NRA], rows_b[NRB];
-        auto load_rows = [&](int32_t b) {
-          if (group_a) {
-#pragma unroll
-            for (int q = 0; q < NRA; ++q) rows_a[q] = row_of(b, own0 + static_cast<int32_t>(r0) + RS * q);
-          } else {
-#pragma unroll
-            for (int q = 0; q < NRB; ++q) rows_b[q] = row_of(b, static_cast<int32_t>(r0) + RS * q);
+        if constexpr (kDense) {
+          // ---- masked dense mode: thread 0 of the group loads each block of its ring with TMA
+          // tile copies into the same swizzled layout, then (one stage behind, so that two stages
+          // are in flight) announces it to the even CTA for the group's four warps at once
+          if (gtid == 0) {
+            const int32_t row0 = (qi / p.n_q) * p.max_len;     // the sequence's first cache row
+            const uint32_t bytes = group_a ? static_cast<uint32_t>(C::SB_BYTES) : static_cast<uint32_t>(C::VR_BYTES);
+            int32_t pend = -1;
+            uint32_t pend_ph = 0;
+            int32_t inflight[2] = {-1, -1};                      // issued stages not yet waited on
+            uint32_t inflight_ph[2] = {0, 0};
+            auto land_and_announce = [&](int32_t stage, uint32_t par) -> bool {
+              const uint32_t tb = group_a ? sb_tma(stage) : vr_tma(stage);
+              if (!wt.wait(tb, par, 15)) return false;
+              if (inflight[0] == stage) inflight[0] = -1;
+              if (inflight[1] == stage) inflight[1] = -1;
+              mbar_arrive_cluster_n(at_leader(group_a ? sb_full2(stage) : vr_full2(stage)),
+                                    static_cast<uint32_t>(C::GROUP_WARPS));
+              return true;
+            };
+            for (int32_t b = 0; b < n_blocks && ok; ++b) {
+              const uint32_t empty_bar = group_a ? sb_empty(st) : vr_empty(st);
+              if (!wt.wait(empty_bar, ph ^ 1u, 11)) { ok = false; break; }
+              const uint32_t tb = group_a ? sb_tma(st) : vr_tma(st);
+              mbar_expect_tx(tb, bytes);
+              if (group_a) {
+                const uint32_t dst = sbase + C::OFF_SB + st * C::SB_BYTES;
+                const int32_t y = row0 + b * kBlk + 32 * static_cast<int32_t>(rank);
+#pragma unroll 1
+                for (int a = 0; a < 9; ++a) tma_load_3d(dst + a * C::SB_ATOM, &map_kv_a, tb, 64 * a, y, 0);
+              } else {
+                const uint32_t dst = sbase + C::OFF_VR + st * C::VR_BYTES;
+                const int32_t y = row0 + b * kBlk;
+                const int32_t x0 = 128 * static_cast<int32_t>(rank);
+                tma_load_3d(dst + 0 * C::VR_ATOM, &map_kv_b, tb, x0 + 0, y, 0);
+                tma_load_3d(dst + 1 * C::VR_ATOM, &map_kv_b, tb, x0 + 64, y, 0);
+                tma_load_3d(dst + 2 * C::VR_ATOM, &map_kv_b, tb, x0 + 256, y, 0);
+                tma_load_3d(dst + 3 * C::VR_ATOM, &map_kv_b, tb, x0 + 320, y, 0);
+              }
+              if (inflight[0] < 0) { inflight[0] = static_cast<int32_t>(st); inflight_ph[0] = ph; }
+              else { inflight[1] = static_cast<int32_t>(st); inflight_ph[1] = ph; }
+              if (pend >= 0 && !land_and_announce(pend, pend_ph)) { ok = false; break; }
+              pend = static_cast<int32_t>(st);
+              pend_ph = ph;
+              if (++st == n_stages) { st = 0; ph ^= 1u; }
+            }
+            if (ok && pend >= 0 && !land_and_announce(pend, pend_ph)) ok = false;
+            // after an abort, every issued copy lands before the CTA may leave
+            for (int k2 = 0; k2 < 2; ++k2)
+              if (inflight[k2] >= 0)
+                attn_drain_wait(group_a ? sb_tma(inflight[k2]) : vr_tma(inflight[k2]), inflight_ph[k2],
+                                kDrainBudgetNs);
           }
-        };
-        load_rows(0);
-        int32_t pending = -1;
-        auto announce = [&](int32_t stage) {
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(at_leader(group_a ? sb_full2(stage) : vr_full2(stage)));
-        };
-        for (int32_t b = 0; b < n_blocks && ok; ++b) {
-          const uint32_t empty_bar = group_a ? sb_empty(st) : vr_empty(st);
-          if (pending >= 0) {                          // about to wait: announce the last stage first
-            uint32_t free_now = 0;
-            if (lane == 0) free_now = mbar_test_wait(empty_bar, ph ^ 1u) ? 1u : 0u;
-            if (!__shfl_sync(0xffffffffu, free_now, 0)) {
-              cp_async_wait<0>();
+        } else {
+          // ---- the ring of this group. Thread (r0, cc) copies 16-byte chunk cc of every 128-byte
+          // segment of block rows r0, r0 + GROUP_THREADS/8, ...: the row indices are read once per block and each
+          // copy is a constant offset from the row's base, so copies issue back to back.
+          const __nv_bfloat16* kv_seq = p.kv + static_cast<size_t>(qi / p.n_q) * p.max_len * kDqk;
+          const uint32_t cc = gtid & 7u, r0 = gtid >> 3;
+          const int32_t own0 = 32 * static_cast<int32_t>(rank);
+          const uint32_t seg0 = 128u * rank;               // group B: segments 2r, 2r+1, 4+2r, 5+2r
+          // block row r of block b: its row of the latent cache, or -1 when masked (padding, past the
+          // extent, or out of range); read from the index row one block ahead of its gathers
+          constexpr int RS = C::GROUP_THREADS / 8;       // rows per pass
+          constexpr int NRA = 32 / RS, NRB = kBlk / RS;  // rows per thread: logits ring, output ring
+          auto row_of = [&](int32_t b, int32_t r) -> int32_t {
+            const int32_t j = b * kBlk + r;
+            const int32_t v = j < total ? __ldg(idx_row + j) : -1;
+            return (v >= 0 && v < p.max_len) ? v : -1;
+          };
+          int32_t rows_a[NRA], rows_b[NRB];
+          auto load_rows = [&](int32_t b) {
+            if (group_a) {
+#pragma unroll
+              for (int q = 0; q < NRA; ++q) rows_a[q] = row_of(b, own0 + static_cast<int32_t>(r0) + RS * q);
+            } else {
+#pragma unroll
+              for (int q = 0; q < NRB; ++q) rows_b[q] = row_of(b, static_cast<int32_t>(r0) + RS * q);
+            }
+          };
+          load_rows(0);
+          int32_t pending = -1;
+          auto announce = [&](int32_t stage) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(at_leader(group_a ? sb_full2(stage) : vr_full2(stage)));
+          };
+          for (int32_t b = 0; b < n_blocks && ok; ++b) {
+            const uint32_t empty_bar = group_a ? sb_empty(st) : vr_empty(st);
+            if (pending >= 0) {                          // about to wait: announce the last stage first
+              uint32_t free_now = 0;
+              if (lane == 0) free_now = mbar_test_wait(empty_bar, ph ^ 1u) ? 1u : 0u;
+              if (!__shfl_sync(0xffffffffu, free_now, 0)) {
+                cp_async_wait<0>();
+                announce(pending);
+                pending = -1;
+              }
+            }
+            if (!warp_wait(empty_bar, ph ^ 1u, 11)) { ok = false; break; }
+            if (group_a) {
+              const uint32_t dst0 = sbase + C::OFF_SB + st * C::SB_BYTES + sw128_offset(r0, cc);
+#pragma unroll
+              for (int q = 0; q < NRA; ++q) {
+                const bool v = rows_a[q] >= 0;
+                const __nv_bfloat16* src = (v ? kv_seq + static_cast<size_t>(rows_a[q]) * kDqk : p.kv) + cc * 8;
+                const uint32_t n = v ? 16u : 0u;
+#pragma unroll
+                for (int a = 0; a < 9; ++a) cp_async_16(dst0 + q * RS * 128 + a * C::SB_ATOM, src + a * 64, n);
+              }
+            } else {
+              const uint32_t dst0 = sbase + C::OFF_VR + st * C::VR_BYTES + sw128_offset(r0, cc);
+#pragma unroll
+              for (int q = 0; q < NRB; ++q) {
+                const bool v = rows_b[q] >= 0;
+                const __nv_bfloat16* src = (v ? kv_seq + static_cast<size_t>(rows_b[q]) * kDqk : p.kv) + seg0 + cc * 8;
+                const uint32_t n = v ? 16u : 0u;
+                const uint32_t d = dst0 + q * RS * 128;
+                cp_async_16(d + 0 * C::VR_ATOM, src + 0, n);
+                cp_async_16(d + 1 * C::VR_ATOM, src + 64, n);
+                cp_async_16(d + 2 * C::VR_ATOM, src + 256, n);
+                cp_async_16(d + 3 * C::VR_ATOM, src + 320, n);
+              }
+            }
+            cp_async_commit();
+            if (b + 1 < n_blocks) load_rows(b + 1);
+            if (pending >= 0) {
+              cp_async_wait<1>();
               announce(pending);
-              pending = -1;
             }
+            pending = static_cast<int32_t>(st);
+            if (++st == n_stages) { st = 0; ph ^= 1u; }
           }
-          if (!warp_wait(empty_bar, ph ^ 1u, 11)) { ok = false; break; }
-          if (group_a) {
-            const uint32_t dst0 = sbase + C::OFF_SB + st * C::SB_BYTES + sw128_offset(r0, cc);
-#pragma unroll
-            for (int q = 0; q < NRA; ++q) {
-              const bool v = rows_a[q] >= 0;
-              const __nv_bfloat16* src = (v ? kv_seq + static_cast<size_t>(rows_a[q]) * kDqk : p.kv) + cc * 8;
-              const uint32_t n = v ? 16u : 0u;
-#pragma unroll
-              for (int a = 0; a < 9; ++a) cp_async_16(dst0 + q * RS * 128 + a * C::SB_ATOM, src + a * 64, n);
-            }
-          } else {
-            const uint32_t dst0 = sbase + C::OFF_VR + st * C::VR_BYTES + sw128_offset(r0, cc);
-#pragma unroll
-            for (int q = 0; q < NRB; ++q) {
-              const bool v = rows_b[q] >= 0;
-              const __nv_bfloat16* src = (v ? kv_seq + static_cast<size_t>(rows_b[q]) * kDqk : p.kv) + seg0 + cc * 8;
-              const uint32_t n = v ? 16u : 0u;
-              const uint32_t d = dst0 + q * RS * 128;
-              cp_async_16(d + 0 * C::VR_ATOM, src + 0, n);
-              cp_async_16(d + 1 * C::VR_ATOM, src + 64, n);
-              cp_async_16(d + 2 * C::VR_ATOM, src + 256, n);
-              cp_async_16(d + 3 * C::VR_ATOM, src + 320, n);
-            }
-          }
-          cp_async_commit();
-          if (b + 1 < n_blocks) load_rows(b + 1);
-          if (pending >= 0) {
-            cp_async_wait<1>();
-            announce(pending);
-          }
-          pending = static_cast<int32_t>(st);
-          if (++st == n_stages) { st = 0; ph ^= 1u; }
+          cp_async_wait<0>();
+          if (pending >= 0) announce(pending);
         }
-        cp_async_wait<0>();
-        if (pending >= 0) announce(pending);
       }
       if (!group_a) {                                  // info[slot] no longer read by this warp
         __syncwarp();
@@ -502,7 +615,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         ++qq;
       }
       tc_commit(mma_done);
-      attn_drain_wait(mma_done, 0, p.wait_budget_ns);
+      attn_drain_wait(mma_done, 0, kDrainBudgetNs);
     } else if (!leader && warp == C::MMA_WARP && lane == 0) {
       // relay of the odd CTA: its softmax warps announce P locally (a CTA-scope arrive does not
       // stall them); this thread observes that (acquire) and forwards one cluster-scope release
@@ -575,10 +688,21 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap map_q, const AttnPara
         const int32_t j = b * kBlk + 32 * static_cast<int32_t>(half) + static_cast<int32_t>(lane);
         return j < total ? __ldg(idx_row + j) : -1;
       };
-      int32_t e_next = entry(0);
+      // masked dense mode: the bitmap word of this half of block b (bit j: position 64b + 32 half
+      // + j is attended; bits at or past the extent are 0)
+      const uint32_t* mask_row = kDense ? p.mask + static_cast<size_t>(qi) * p.mask_words : nullptr;
+      auto mask_word = [&](int32_t b) -> uint32_t { return __ldg(mask_row + 2 * b + static_cast<int32_t>(half)); };
+      int32_t e_next = kDense ? 0 : entry(0);
+      uint32_t m_next = kDense ? mask_word(0) : 0u;
       for (int32_t b = 0; b < n_blocks && ok; ++b) {
-        const uint32_t vmask = __ballot_sync(0xffffffffu, e_next >= 0 && e_next < p.max_len);
-        if (b + 1 < n_blocks) e_next = entry(b + 1);
+        uint32_t vmask;
+        if constexpr (kDense) {
+          vmask = m_next;
+          if (b + 1 < n_blocks) m_next = mask_word(b + 1);
+        } else {
+          vmask = __ballot_sync(0xffffffffu, e_next >= 0 && e_next < p.max_len);
+          if (b + 1 < n_blocks) e_next = entry(b + 1);
+        }
         // ---- this lane's 32 logits
         if (lane == 0) got = wt.wait(s_full(s_i), s_u & 1u, 32) ? 1u : 0u;
         if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }

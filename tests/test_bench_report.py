@@ -82,3 +82,27 @@ def test_row_sharded_line_is_strong_scaling_over_the_whole_sequence():
     assert line["stages"]["allgather"]["bytes"] == cfg.max_len * (128 + 4 + 576 * 2)
     w0 = bench._work_rows(cfg, *parts[0])
     assert line["stages"]["indexer_topk"]["achieved"] == pytest.approx(w0["indexer_flop"] / 1.2e-3 / 1e12)
+
+
+def test_torchrun_command_runs_this_bench_as_n_local_ranks():
+    cmd = bench.torchrun_command(4, ["--gpus", "4", "--steps", "3"], 29512)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--master-addr=127.0.0.1" in cmd and "--master-port=29512" in cmd
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "3"] and cmd[-5].endswith("bench.py")
+
+
+def test_gpus_2_spawns_two_ranks_with_their_environment():
+    # `bench.py --gpus 2` outside torchrun relaunches itself as two ranks; --print-ranks makes each
+    # rank report its environment and exit before touching a GPU
+    import json
+    import os
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    out = subprocess.run([sys.executable, os.path.abspath(bench.__file__), "--gpus", "2", "--print-ranks"],
+                         capture_output=True, text=True, timeout=240, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    ranks = [json.loads(line) for line in out.stdout.splitlines() if line.startswith("{")]
+    assert sorted(r["RANK"] for r in ranks) == ["0", "1"]
+    assert all(r["WORLD_SIZE"] == "2" and r["MASTER_ADDR"] == "127.0.0.1" for r in ranks)
+    assert sorted(r["LOCAL_RANK"] for r in ranks) == ["0", "1"]

@@ -169,6 +169,39 @@ def test_equal_scores_select_the_lowest_positions():
         assert (idx_h[i, n:] == -1).all()
 
 
+def test_sampled_threshold_falls_back_to_the_exact_pass():
+    """Queries long enough for the sampled threshold (>= 64 key tiles). In every other block of
+    four queries all index scores are 0 (w = 0): the sample phase then drops candidates that tie
+    for their position, so those items must be rerun exactly and keep the lowest 2048
+    positions; the other items keep their sampled selection, checked against the oracle."""
+    cfg = synthetic.config("prefill_4k", n_q=9000, max_len=9000)
+    g = {}
+    g["q_idx"], g["q_scale"] = synthetic.gen_q_idx(cfg, 17, "cuda")
+    g["k_idx"], g["k_scale"] = synthetic.gen_k_idx(cfg, 17, "cuda")
+    g["w"] = synthetic.gen_w(cfg, 17, "cuda")
+    zero = torch.arange(cfg.n_q, device="cuda") // 4 % 2 == 0
+    g["w"][zero] = 0
+    dims = dsa.dims_for(cfg)
+    ws = dsa.Workspace.create(dims, cfg.topk)
+    idx = dsa.indexer_topk(dims, g["q_idx"].view(1, cfg.n_q, cfg.n_idx_heads, cfg.idx_dim),
+                           g["w"].view(1, cfg.n_q, -1), g["k_idx"], g["q_scale"], g["k_scale"],
+                           synthetic.lengths(cfg, 17).cuda(), cfg.topk, ws)
+    torch.cuda.synchronize()
+    ws.check()
+    idx_h = idx.cpu().numpy()[0]
+    zero_h = zero.cpu().numpy()
+    for i in range(8000, cfg.n_q):                   # positions of at least 8064 use the sample phase
+        if zero_h[i]:
+            assert sorted(idx_h[i, :cfg.topk].tolist()) == list(range(cfg.topk)), f"row {i}"
+    ro = RowOracle(cfg, 17)
+    rows = [i for i in synthetic.sample_rows(cfg.n_q, 40, 17, extra=[8063, 8064, 8999]) if not zero_h[i]]
+    stats = []
+    for j, i in enumerate(rows):
+        _, scores = ro.indexer(0, i)
+        stats.append(check_selection(idx_h[i], scores, cfg.topk, i))
+    report_near_ties("prefill L=9000, sampled threshold", len(rows), stats)
+
+
 def test_decode_equal_scores_merge_by_position():
     # every index score is 0, so each sequence keeps its lowest min(k, len) positions; with
     # lengths spanning one to three 8192-key chunks, the merge must resolve the ties across
