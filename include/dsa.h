@@ -86,8 +86,10 @@ dsa_status dsa_workspace_init(void* ws, size_t ws_bytes, dsa_stream_t stream);
  *   out_idx int32    [B, n_q, topk]: positions s <= pos of the min(topk, pos+1) largest
  *           scores of each query, in unspecified order, then -1 padding. Ties between equal
  *           scores go to the lower position.
- * The L x L score matrix is never stored: scores stream from the tensor cores into a running
- * per-query selection in shared memory.
+ * Prefill (n_q > 1) never stores the L x L score matrix: scores stream from the tensor cores
+ * into a running per-query selection in shared memory. Decode (n_q = 1) with max_len <= 131072
+ * writes each sequence's single score row (4 B per key) to the workspace and selects from it;
+ * longer decode rows keep a partial top-k per 8192-key chunk in the workspace and merge them.
  */
 dsa_status dsa_indexer_topk(const dsa_dims* dims, const void* q_idx, const void* w, const void* k_idx,
                             const float* scales, const int32_t* lengths, int32_t topk, int32_t* out_idx,

@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdsa.so")
 SOURCES = ["dsa_api.cu"]
-HEADERS = ["ptx.cuh", "select.cuh", "indexer_topk.cuh", "sparse_mla.cuh"]
+HEADERS = ["ptx.cuh", "select.cuh", "indexer_topk.cuh", "decode_select.cuh", "sparse_mla.cuh", "indexer_kl.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -12,6 +12,7 @@
 
 #include "dsa.h"
 #include "indexer_topk.cuh"
+#include "decode_select.cuh"
 #include "sparse_mla.cuh"
 #include "indexer_kl.cuh"
 
@@ -113,7 +114,8 @@ dsa_status check_dims(const dsa_dims* d, int32_t topk) {
 // Workspace regions, each 256-byte aligned.
 struct Layout {
   size_t status = 0;                     // 256 B: status word + detail
-  size_t part_keys = 0, part_pos = 0, part_count = 0;   // decode partial top-k
+  size_t key_rows = 0;                   // decode: every key of the row (max_len <= kSelMaxLen)
+  size_t part_keys = 0, part_pos = 0, part_count = 0;   // decode beyond that: partial top-k
   size_t redo_flag = 0, redo_list = 0, redo_count = 0;  // prefill items queued for the exact pass
   size_t idx = 0;                        // forward's selection when out_idx == NULL
   size_t mask = 0, extent = 0;           // masked dense mode: bitmap rows and extents
@@ -133,10 +135,14 @@ Layout make_layout(const dsa_dims& d, int32_t topk) {
   const int64_t K = static_cast<int64_t>(d.batch) * d.max_len;
   if (d.n_q == 1) {
     L.n_chunks = (d.max_len + kDecodeChunk - 1) / kDecodeChunk;
-    const size_t slots = static_cast<size_t>(d.batch) * L.n_chunks;
-    L.part_keys = off; off = align_up(off + slots * topk * 4);
-    L.part_pos = off; off = align_up(off + slots * topk * 4);
-    L.part_count = off; off = align_up(off + slots * 4);
+    if (d.max_len <= kSelMaxLen) {
+      L.key_rows = off; off = align_up(off + static_cast<size_t>(K) * 4);
+    } else {
+      const size_t slots = static_cast<size_t>(d.batch) * L.n_chunks;
+      L.part_keys = off; off = align_up(off + slots * topk * 4);
+      L.part_pos = off; off = align_up(off + slots * topk * 4);
+      L.part_count = off; off = align_up(off + slots * 4);
+    }
   }
   if (sampled_threshold(d, topk)) {
     const size_t items = static_cast<size_t>(d.batch) * ((d.n_q + kPrefillNQ - 1) / kPrefillNQ);
@@ -316,10 +322,18 @@ dsa_status run_indexer(const dsa_dims& d, const uint8_t* q_idx, const __nv_bfloa
   if (!encode_rows_u8(&map_k, k_idx, static_cast<uint64_t>(d.max_len), static_cast<uint64_t>(d.batch), kKeyTile))
     return DSA_ERR_CUDA;
   if (d.n_q == 1) {
+    // decode: the chunk items score every key of the row; rows up to kSelMaxLen keys are then
+    // selected whole by one cluster per sequence, longer ones keep a partial top-k per chunk
+    // that a merge reduces
+    const bool rows = L.key_rows != 0;
     p.n_chunks = L.n_chunks;
-    p.part_keys = reinterpret_cast<uint32_t*>(ws + L.part_keys);
-    p.part_pos = reinterpret_cast<int32_t*>(ws + L.part_pos);
-    p.part_count = reinterpret_cast<int32_t*>(ws + L.part_count);
+    if (rows) {
+      p.key_rows = reinterpret_cast<uint32_t*>(ws + L.key_rows);
+    } else {
+      p.part_keys = reinterpret_cast<uint32_t*>(ws + L.part_keys);
+      p.part_pos = reinterpret_cast<int32_t*>(ws + L.part_pos);
+      p.part_count = reinterpret_cast<int32_t*>(ws + L.part_count);
+    }
     p.n_items = d.batch * L.n_chunks;
     if (!encode_rows_u8(&map_q, q_idx, static_cast<uint64_t>(kIdxHeads), static_cast<uint64_t>(d.batch),
                         kIdxHeads))
@@ -328,8 +342,13 @@ dsa_status run_indexer(const dsa_dims& d, const uint8_t* q_idx, const __nv_bfloa
     indexer_topk_kernel<1><<<grid, IdxCfg<1>::THREADS, IdxCfg<1>::SMEM_BYTES, st>>>(map_q, map_k, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return DSA_ERR_CUDA;
-    MergeParams mp{p.part_keys, p.part_pos, p.part_count, out_idx, L.n_chunks, topk, out_scores};
-    merge_partials_kernel<kMergeThreads><<<d.batch, kMergeThreads, 0, st>>>(mp);
+    if (rows) {
+      DecodeSelectParams sp{p.key_rows, lengths, out_idx, out_scores, d.max_len, topk};
+      decode_select_kernel<<<d.batch * kSelCluster, kSelThreads, 0, st>>>(sp);
+    } else {
+      MergeParams mp{p.part_keys, p.part_pos, p.part_count, out_idx, L.n_chunks, topk, out_scores};
+      merge_partials_kernel<kMergeThreads><<<d.batch, kMergeThreads, 0, st>>>(mp);
+    }
     return from_cuda(cudaGetLastError());
   }
   p.n_chunks = 0;

@@ -30,9 +30,9 @@
 //    admission threshold for the other tiles, which then follow in position order. About 1.5 k
 //    keys of the whole range score at least that, so the candidate buffers rarely need a shrink
 //    afterwards. The threshold is a guess, so the item checks it: if a query ends with fewer
-//    than k candidates, or the sample phase dropped candidates that tied with the k-th for
-//    their position, the item is queued and a second launch reruns the queued items with the
-//    exact streaming threshold. Thresholds in a sampled item never exclude ties (the stream is
+//    than k candidates, or its sample phase had to cut a group of equal keys too large to keep
+//    (the sample phase otherwise keeps every key tied with its r-th), the item is queued and a
+//    second launch reruns the queued items with the exact streaming threshold. Thresholds in a sampled item never exclude ties (the stream is
 //    not in position order), so the final selection settles ties by position as always.
 #pragma once
 #include <cstdint>
@@ -47,11 +47,10 @@ constexpr int kIdxHeads = 64;     // H_I (padded)
 constexpr int kIdxDim = 128;      // d_I (padded), one 128-byte row per head / key
 constexpr int kKeyTile = 128;     // keys per MMA tile (M)
 constexpr int kDecodeChunk = 8192;  // keys per decode work item
-constexpr int kSyncTiles = 8;       // key tiles between two capacity checks of a candidate buffer
 constexpr int kSampleStride = 16;   // sampled threshold: the sample is every 16th key tile
 constexpr int kSpecMinTiles = 64;   // ... for items with at least this many key tiles
 constexpr int kSpecMinTopk = 1024;  // ... and at least this top-k (the sample's rank is ~ 3 k / 32)
-constexpr int kSampleLimit = 1024;  // candidate count above which the sample phase shrinks its buffer
+constexpr int kSampleLimit = 2048;  // candidate count above which the sample phase shrinks its buffer
 
 template <int NQ>
 struct IdxCfg {
@@ -83,6 +82,9 @@ struct IdxCfg {
   static constexpr int K_BYTES = kKeyTile * kIdxDim;       // 16 KB
   static constexpr int TMEM_COLS = NBUF * N;
   static constexpr int MAXPER = CAND / GROUP_THREADS;
+  // key tiles between two capacity checks of a candidate buffer (each check is a named barrier
+  // of the query's warps; decode chunks are short, so they check more often)
+  static constexpr int SYNC = (NQ == 4) ? 8 : 4;
   // shared-memory layout (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
@@ -96,7 +98,8 @@ struct IdxCfg {
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(CAND % GROUP_THREADS == 0 && MAXPER <= 64, "candidate buffer must split evenly");
-  static_assert(CAND - kSyncTiles * kKeyTile >= 2048, "a checked buffer must hold the largest k");
+  static_assert(CAND - SYNC * kKeyTile >= 2048, "a checked buffer must hold the largest k");
+  static_assert(kSampleLimit + SYNC * kKeyTile <= CAND, "sample-phase limit");
   static_assert(NBUF * HALVES <= 4 && TMEM_COLS <= 512, "accumulators");
   static_assert(THREADS <= 1024 && NQ <= 4, "block shape");
   // setmaxnreg.inc waits until the registers the block was launched with can serve it, so the
@@ -118,6 +121,9 @@ struct IndexerParams {
   uint32_t* part_keys;      // decode: [B, n_chunks, topk]
   int32_t* part_pos;        // decode: [B, n_chunks, topk]
   int32_t* part_count;      // decode: [B, n_chunks]
+  // decode, score-only: when set, every key's order-preserving score goes to key_rows
+  // [B, max_len] (positions the query sees) and no selection is made here
+  uint32_t* key_rows;
   uint32_t* status;
   int32_t batch, n_q, max_len, topk, n_chunks;
   int32_t n_items;
@@ -263,11 +269,11 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
   }
   const int32_t G = gridDim.x;
   const int32_t cta = blockIdx.x;
-  if (NQ == 1 || (p.spec && p.item_list == nullptr)) {
-    // Per-item words that only this CTA writes start at zero here, before the barrier. Decode:
-    // slot u of the partial lists belongs to item u, so a slot this CTA never reaches (after an
+  if ((NQ == 1 && p.part_count != nullptr) || (NQ > 1 && p.spec && p.item_list == nullptr)) {
+    // Per-item words that only this CTA writes start at zero here, before the barrier. Decode
+    // with partial lists: slot u belongs to item u, so a slot this CTA never reaches (after an
     // aborted wait) reads as empty in the merge instead of holding an earlier call's count.
-    // Sampled prefill: item u's queued flag.
+    // (Score-only decode has no per-item words.) Sampled prefill: item u's queued flag.
     for (int32_t r = static_cast<int32_t>(threadIdx.x);; r += static_cast<int32_t>(blockDim.x)) {
       const int32_t u = item_of(r, cta, G);
       if (u >= p.n_items) break;
@@ -498,7 +504,11 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
               (((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y))) * ks;
           key = score_key(score);
           const bool valid = in_range && s <= qpos;
-          pass = valid && (key > thr_r || (key == thr_r && strict_r == 0));
+          if (NQ == 1 && p.key_rows != nullptr) {
+            if (valid) p.key_rows[static_cast<size_t>(it.b) * p.max_len + s] = key;
+          } else {
+            pass = valid && (key > thr_r || (key == thr_r && strict_r == 0));
+          }
         }
         // this tile's passes go into the buffer at once: one ballot, and one atomic for a warp
         // with any pass (after the first few tiles most warps have none)
@@ -513,65 +523,79 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
             cq_pos[at] = s;
           }
         }
-        // capacity check every kSyncTiles tiles: between two checks at most kSyncTiles * 128
-        // candidates arrive, and a check leaves at most CAND - kSyncTiles * 128 (also at the
+        // capacity check every C::SYNC tiles: between two checks at most C::SYNC * 128
+        // candidates arrive, and a check leaves at most CAND - C::SYNC * 128 (also at the
         // end of a sample phase)
         const bool boundary = t + 1 == it.n_s;
-        if (t % kSyncTiles != kSyncTiles - 1 && t + 1 != it.ntiles && !boundary) continue;
+        if (t % C::SYNC != C::SYNC - 1 && t + 1 != it.ntiles && !boundary) continue;
         if (uniform_stop()) { stop = true; break; }
+        if (NQ == 1 && p.key_rows != nullptr) continue;
         uint32_t n = q_count[q];
         // the sample phase selects the sample's r best, under a lower capacity limit
         const bool sampling = t < it.n_s;
         const uint32_t tgt = sampling ? sample_rank(p.topk, it) : static_cast<uint32_t>(p.topk);
         const uint32_t limit = sampling ? static_cast<uint32_t>(kSampleLimit)
-                                        : static_cast<uint32_t>(C::CAND - kSyncTiles * kKeyTile);
+                                        : static_cast<uint32_t>(C::CAND - C::SYNC * kKeyTile);
+        // Beyond the cheap shrink, a check may keep the tgt best with every candidate tied with
+        // the tgt-th (the sample phase: a tie dropped there could still belong to the final
+        // top-k; and the end of the sample phase, whose r-th key becomes the threshold), or
+        // select exactly tgt, cutting ties by position (streaming, or a sample-phase tie group
+        // too large to keep, after which the item is rerun exactly).
+        bool keep = boundary, exact = false;
         if (n > limit) {
-          // cheap range-histogram shrink; the exact select only if it frees too little
           uint32_t thr = 0;
           const uint32_t m = shrink_candidates<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, n, tgt, gsel, gtid,
                                                                             bar_id, &thr);
-          // the exact select when the shrink freed less than half of the usable space
+          // more when the shrink freed less than half of the usable space
           if (m > (limit + tgt) / 2) {
-            bool tied = false;
-            const uint32_t vk =
-                select_exact<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, m, tgt, gsel, gtid, bar_id, &tied);
-            if (sampling && tied) sample_tie = true;
-            if (gtid == 0) {
-              q_count[q] = tgt;
-              q_thr[q] = vk;
-              // a strict threshold relies on later keys having larger positions: only in
-              // position order
-              q_strict[q] = it.n_s == 0 ? 1u : 0u;
-            }
-          } else if (gtid == 0) {
+            keep = keep || sampling;
+            exact = !sampling;
+          }
+          if (gtid == 0) {
             q_count[q] = m;
             q_thr[q] = thr;
             q_strict[q] = 0;
           }
           named_barrier(bar_id, C::GROUP_THREADS);
           thr_r = q_thr[q];
-          strict_r = q_strict[q];
+          strict_r = 0;
           n = q_count[q];
         }
-        if (boundary && n > tgt) {
-          // end of the sample phase: the sample's r-th best key becomes the admission threshold
-          // (non-strict); every candidate at or above it stays
+        if (keep && n > tgt) {
           uint32_t kept = 0;
           const uint32_t v =
               select_keep_ge<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, n, tgt, gsel, gtid, bar_id, &kept);
-          if (gtid == 0) {
+          if (kept > (limit + tgt) / 2) {
+            exact = true;
+          } else if (gtid == 0) {
             q_count[q] = kept;
             q_thr[q] = max(v, thr_r);
             q_strict[q] = 0;
           }
           named_barrier(bar_id, C::GROUP_THREADS);
           thr_r = q_thr[q];
-          strict_r = 0;
+          n = exact ? kept : q_count[q];
+        }
+        if (exact) {
+          bool tied = false;
+          const uint32_t vk =
+              select_exact<C::GROUP_THREADS, C::MAXPER>(cq_keys, cq_pos, n, tgt, gsel, gtid, bar_id, &tied);
+          if (sampling && tied) sample_tie = true;
+          if (gtid == 0) {
+            q_count[q] = tgt;
+            q_thr[q] = vk;
+            // a strict threshold relies on later keys having larger positions: only in
+            // position order
+            q_strict[q] = it.n_s == 0 ? 1u : 0u;
+          }
+          named_barrier(bar_id, C::GROUP_THREADS);
+          thr_r = q_thr[q];
+          strict_r = q_strict[q];
         }
       }
       if (stop) break;
       // ---- finish the query: exact k, then write
-      if (q_valid) {
+      if (q_valid && !(NQ == 1 && p.key_rows != nullptr)) {
         uint32_t n = q_count[q];
         // a sampled item whose threshold kept fewer than k candidates, or dropped ties in its
         // sample phase, is queued for the exact pass (which rewrites all its queries)

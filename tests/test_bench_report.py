@@ -52,6 +52,13 @@ def test_decode_line_is_hbm_bound_in_sequences_per_second():
     assert line["roofline"]["kernel"] == "indexer_topk"
 
 
+def test_other_prefill_workloads_name_their_own_sizes():
+    cfg = synthetic.config("prefill_4k")
+    line = bench.report(_args(), cfg, _res(2), 1)
+    assert line["metric"] == "DSA prefill query-tokens/s (indexer+top-k+sparse MLA) at L=4096, k=2048"
+    assert line["unit"] == "query-tokens/s"
+
+
 def test_prefill_line_keeps_the_headline_metric():
     cfg = synthetic.config("prefill_128k")
     line = bench.report(_args(), cfg, _res(2), 1)

@@ -219,6 +219,81 @@ def test_decode_equal_scores_merge_by_position():
         assert (idx_h[b, 0, n:] == -1).all()
 
 
+def test_decode_repeated_keys_cut_ties_by_position():
+    """Cached index keys repeat with period 97, so each sequence's scores take 97 values, each
+    held by many positions: the k-th score is shared by more positions than places remain,
+    and the selection must keep the lowest of them. The oracle ranks the same way (score,
+    then position), so the selected sets must be equal; the premise (the k-th score well
+    apart from the scores next to it, its group split) is checked on the oracle's scores first."""
+    period = 97
+    cfg = synthetic.config("decode", batch=3, max_len=30000, len_range=(100, 30000))
+    g = _inputs(cfg, 21)
+    lens = [30000, 12345, 4100]
+    g["lengths"] = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    rep = torch.arange(cfg.max_len, device="cuda") % period
+    g["k_idx"] = g["k_idx"][:, rep].contiguous()
+    g["k_scale"] = g["k_scale"][:, rep].contiguous()
+    idx, out, lse = _run_forward(cfg, g)
+    idx_h = idx.cpu().numpy()
+    ro = RowOracle(cfg, 21, lengths=torch.tensor(lens))
+    for b, n_b in enumerate(lens):
+        kc, ks = synthetic.gen_k_idx(cfg, 21, b=b, s_range=range(0, period))
+        rep_h = np.arange(n_b) % period
+        ro._keys[b] = (kc.numpy()[rep_h], ks.numpy()[rep_h])
+        sel_o, scores = ro.indexer(b, 0)
+        distinct = np.unique(scores)[::-1]
+        assert len(distinct) == period
+        kth = np.sort(scores)[::-1][cfg.topk - 1]
+        at = int(np.flatnonzero(distinct == kth)[0])
+        gaps = np.array([distinct[at - 1] - kth, kth - distinct[at + 1]])
+        assert (gaps > 1e-4 * np.max(np.abs(distinct))).all()             # far above fp32 rounding
+        assert (scores > kth).sum() < cfg.topk < (scores >= kth).sum()       # the k-th group is split
+        assert sorted(idx_h[b, 0].tolist()) == sorted(sel_o.tolist()), f"sequence {b}"
+
+
+def test_decode_select_falls_back_when_the_sample_misleads():
+    """The decode select guesses a threshold from a 1/16 sample of the row: the key slots at
+    positions p with p mod 4096 < 256. Here the first 300 sampled positions carry the row's best
+    key at twice its scale, so the sample's r-th key (r ~ 200) is one of them and only those 300
+    keys reach it, fewer than k. The select must notice and run over the whole row; the result
+    is checked against the oracle on the same modified inputs."""
+    cfg = synthetic.config("decode", batch=2, max_len=40000, len_range=(4096, 40000))
+    g = _inputs(cfg, 25)
+    lens = [40000, 30000]
+    g["lengths"] = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    ro = RowOracle(cfg, 25, lengths=torch.tensor(lens))
+    strong = {}
+    for b, n_b in enumerate(lens):
+        _, sc = ro.indexer(b, 0)
+        best = int(np.argmax(sc))
+        assert sc[best] > 0
+        s = np.flatnonzero(np.arange(n_b) % 4096 < 256)[:300]
+        kc, ks = (a.copy() for a in ro.keys(b))
+        kc[s], ks[s] = kc[best], ks[best] * 2
+        ro._keys[b] = (kc, ks)
+        st = torch.from_numpy(s).cuda()
+        g["k_idx"][b, st] = g["k_idx"][b, best].clone()
+        g["k_scale"][b, st] = g["k_scale"][b, best].clone() * 2
+        strong[b] = set(s.tolist())
+    idx, out, lse = _run_forward(cfg, g)
+    _check_rows(cfg, 25, [(0, 0), (1, 0)], idx, out, lse, ro=ro, name="decode, misleading sample")
+    idx_h = idx.cpu().numpy()
+    for b in range(cfg.batch):
+        assert strong[b] <= set(idx_h[b, 0].tolist())
+
+
+def test_decode_rows_longer_than_one_select_cluster():
+    """Decode rows of more than 131072 keys take the per-chunk partial top-k and its merge
+    instead of the whole-row select; checked against the oracle like the decode workload."""
+    cfg = synthetic.config("decode", batch=2, max_len=140000, len_range=(4096, 140000))
+    g = _inputs(cfg, 23)
+    lens = torch.tensor([140000, 70001], dtype=torch.int32)
+    g["lengths"] = lens.cuda()
+    idx, out, lse = _run_forward(cfg, g)
+    ro = RowOracle(cfg, 23, lengths=lens)
+    _check_rows(cfg, 23, [(0, 0), (1, 0)], idx, out, lse, ro=ro, name="decode, rows of 140000 keys")
+
+
 @pytest.mark.parametrize("topk", [1, 7, 2048])
 def test_topk_extremes(topk):
     cfg = synthetic.config("tiny", n_q=260, max_len=260, topk=topk)
