@@ -539,10 +539,13 @@ def run_e2e_decode(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
     """A decode step end to end through the public API, as a serving loop runs it: the caches
     (indexer keys, their scales and the latent rows) stay resident on the device; every step
     uploads the new queries' inputs and the lengths from pinned host memory and reads back out,
-    lse and idx. Appending the new token's own cache rows belongs to the caller's cache
-    management and is not part of this path."""
+    lse and idx. Successive steps are independent request batches, so they pipeline: a step's
+    inputs go up on a copy stream while the step before computes and the one before that comes
+    back on a second copy stream, through a ring of device buffers. Appending the new token's own
+    cache rows belongs to the caller's cache management and is not part of this path."""
     B = cfg.batch
     q_side = ["q_idx", "w", "q", "lengths"]
+    NS = 3                                               # device buffer slots
     try:
         host = {n: torch.empty(g[n].shape, dtype=g[n].dtype, pin_memory=True) for n in q_side}
         host_qs = torch.empty((B * cfg.n_q,), dtype=torch.float32, pin_memory=True)
@@ -554,23 +557,45 @@ def run_e2e_decode(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
     for n in q_side:
         host[n].copy_(g[n])
     host_qs.copy_(scales[:B * cfg.n_q])
-    dev_in = {n: torch.empty_like(g[n]) for n in q_side}
-    dev_scales = scales.clone()                      # key scales resident; query scales rewritten per step
-    out = torch.empty(host_out.shape, dtype=host_out.dtype, device=dev)
-    lse = torch.empty(host_lse.shape, dtype=host_lse.dtype, device=dev)
-    idx = torch.empty(host_idx.shape, dtype=host_idx.dtype, device=dev)
+    # per slot: the query side, the scales (key scales resident, query scales rewritten per step)
+    # and the outputs
+    slot = [dict({n: torch.empty_like(g[n]) for n in q_side}, scales=scales.clone(),
+                 out=torch.empty(host_out.shape, dtype=host_out.dtype, device=dev),
+                 lse=torch.empty(host_lse.shape, dtype=host_lse.dtype, device=dev),
+                 idx=torch.empty(host_idx.shape, dtype=host_idx.dtype, device=dev)) for _ in range(NS)]
     h2d = sum(host[n].numel() * host[n].element_size() for n in q_side) + host_qs.numel() * 4
     d2h = host_out.numel() * 2 + host_lse.numel() * 4 + host_idx.numel() * 4
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    prev = {"comp": [None] * NS, "d2h": [None] * NS, "n": 0}
 
     def step():
-        for n in q_side:
-            dev_in[n].copy_(host[n], non_blocking=True)
-        dev_scales[:B * cfg.n_q].copy_(host_qs, non_blocking=True)
-        dsa.dsa_forward(dims, dev_in["q_idx"], dev_in["w"], g["k_idx"], dev_scales, dev_in["lengths"], cfg.topk,
-                        dev_in["q"], g["kv"], idx, out, lse, ws.buf, stream)
-        host_out.copy_(out, non_blocking=True)
-        host_lse.copy_(lse, non_blocking=True)
-        host_idx.copy_(idx, non_blocking=True)
+        sl = prev["n"] % NS
+        prev["n"] += 1
+        bufs = slot[sl]
+        with torch.cuda.stream(s_in):
+            if prev["comp"][sl] is not None:
+                s_in.wait_event(prev["comp"][sl])          # the slot's inputs are no longer read
+            for n in q_side:
+                bufs[n].copy_(host[n], non_blocking=True)
+            bufs["scales"][:B * cfg.n_q].copy_(host_qs, non_blocking=True)
+            ready = torch.cuda.Event()
+            ready.record(s_in)
+        stream.wait_event(ready)
+        if prev["d2h"][sl] is not None:
+            stream.wait_event(prev["d2h"][sl])             # the slot's outputs have been read back
+        dsa.dsa_forward(dims, bufs["q_idx"], bufs["w"], g["k_idx"], bufs["scales"], bufs["lengths"], cfg.topk,
+                        bufs["q"], g["kv"], bufs["idx"], bufs["out"], bufs["lse"], ws.buf, stream)
+        done = torch.cuda.Event()
+        done.record(stream)
+        prev["comp"][sl] = done
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done)
+            host_out.copy_(bufs["out"], non_blocking=True)
+            host_lse.copy_(bufs["lse"], non_blocking=True)
+            host_idx.copy_(bufs["idx"], non_blocking=True)
+            back = torch.cuda.Event()
+            back.record(s_out)
+            prev["d2h"][sl] = back
 
     steps = max(3, args.steps)
     for _ in range(3):
@@ -579,16 +604,17 @@ def run_e2e_decode(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):
     if world > 1:
         torch.distributed.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
+    a.record(s_in)
     for _ in range(steps):
         step()
-    b.record(stream)
+    b.record(s_out)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(a.elapsed_time(b), dev)
     ws.check()
     return {"value": aggregate_value(B * cfg.n_q, steps, world, ms), "unit": DECODE_UNIT, "steps": steps,
             "ms_per_step": ms / steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "pinned": True,
-            "caches": "resident on the device (uploaded once, outside the timed region)"}
+            "caches": "resident on the device (uploaded once, outside the timed region)",
+            "streams": "h2d / compute / d2h overlapped across steps (independent request batches)"}
 
 
 def run_e2e(args, cfg, dsa, dims, g, scales, ws, dev, stream, world):

@@ -17,6 +17,12 @@
 // decisions. Keys equal to the k-th are resolved by further passes over their positions
 // (lowest first).
 //
+// Before that, a guess: the r-th best key of a 1/16 sample of the row (r ~ 1.5 k scaled to
+// the sample, as in the indexer's prefill items) is very likely below the k-th key. One stream
+// over the row keeps every key at or above it in shared memory (about 1.5 k for the whole
+// row), and when no CTA overflowed and at least k keys made it, the passes run over those
+// candidates only; otherwise they run over the whole row.
+//
 // Ranking matches select.cuh: key descending, then position ascending. The output row holds
 // min(k, n) positions (in no particular order) followed by -1.
 #pragma once

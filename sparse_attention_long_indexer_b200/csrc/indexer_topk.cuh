@@ -433,10 +433,11 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       const float* ks_row = p.k_scale + static_cast<size_t>(it.b) * p.max_len;
       const int32_t s_lane = it.s_begin + static_cast<int32_t>(quarter * 32 + lane);
       // this lane's key at step t; the next step's key and its scale are fetched one step ahead
-      // (clamped address: the scale of a key past the range is never used)
+      // (address clamped to the item's range: the scale of a key outside it is never used)
       auto key_at = [&](int32_t t) -> int32_t { return s_lane + tile_at(it, t) * kKeyTile; };
+      auto scale_at = [&](int32_t s) -> float { return __ldg(ks_row + max(min(s, it.s_end - 1), 0)); };
       int32_t s_next = key_at(0);
-      float ks_next = __ldg(ks_row + min(s_next, it.s_end - 1));
+      float ks_next = scale_at(s_next);
       // a sampled item may drop candidates that tie with the sample's selection for their
       // position; its queries are then rerun exactly
       bool sample_tie = false;
@@ -446,7 +447,7 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         const int32_t s = s_next;
         const float ks = ks_next;
         s_next = key_at(t + 1);
-        ks_next = __ldg(ks_row + min(s_next, it.s_end - 1));
+        ks_next = scale_at(s_next);
         const bool in_range = s < it.s_end;
         // every lane waits (no divergent branch); the warp then runs the collective TMEM loads
         const bool ok = __all_sync(0xffffffffu, wt.wait(acc_full(buf, half), acc_ph, 8)) != 0;
