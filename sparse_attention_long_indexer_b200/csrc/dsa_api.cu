@@ -10,6 +10,8 @@
 #include <atomic>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "dsa.h"
 #include "indexer_topk.cuh"
 #include "decode_select.cuh"
@@ -74,6 +76,16 @@ __global__ void fill_cols_kernel(T* __restrict__ dst, int64_t rows, int cols_fro
 using namespace dsa;
 
 namespace {
+
+// An NVTX range over a scope: each call and each stage it launches shows up by name in a profiler
+// timeline (`ncu --nvtx --nvtx-include ...` can filter on them). Header-only NVTX3: without a tool
+// attached the calls do nothing.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr uint64_t kWaitBudgetNs = 2000000000ull;   // 2 s per bounded wait
 // budget of the indexer's pipeline waits (dsa_set_wait_budget_ns, a test setting)
@@ -303,6 +315,7 @@ cudaError_t launch_unpad(const T* src, T* dst, int64_t rows, int hs, int ds, int
 dsa_status run_indexer(const dsa_dims& d, const uint8_t* q_idx, const __nv_bfloat16* w, const uint8_t* k_idx,
                        const float* scales, const int32_t* lengths, int32_t topk, int32_t* out_idx,
                        float* out_scores, uint8_t* ws, const Layout& L, cudaStream_t st) {
+  NvtxRange range("indexer_topk");
   const DeviceInfo dev = device_info();
   IndexerParams p{};
   p.q_idx = q_idx;
@@ -385,6 +398,7 @@ dsa_status run_indexer(const dsa_dims& d, const uint8_t* q_idx, const __nv_bfloa
 dsa_status run_attention(const dsa_dims& d, const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
                          int32_t topk, __nv_bfloat16* out, float* lse, uint8_t* ws, const Layout& L,
                          cudaStream_t st, bool masked) {
+  NvtxRange range(masked ? "masked_mqa_attn" : "sparse_mla_attn");
   const DeviceInfo dev = device_info();
   AttnParams p{};
   p.q = q;
@@ -575,6 +589,7 @@ dsa_status dsa_masked_mqa_attn(const dsa_dims* dims, const void* q, const void* 
 dsa_status dsa_indexer_kl_loss(const dsa_dims* dims, const void* q, const void* latent_kv, const int32_t* idx,
                                const float* idx_scores, const float* lse, int32_t topk, float* loss, void* ws,
                                size_t ws_bytes, dsa_stream_t stream) {
+  NvtxRange range("indexer_kl_loss");
   dsa_status s = check_dims(dims, topk);
   if (s != DSA_OK) return s;
   const dsa_dims& d = *dims;
@@ -623,6 +638,7 @@ dsa_status dsa_forward(const dsa_dims* dims, const void* q_idx, const void* w, c
                        const float* scales, const int32_t* lengths, int32_t topk, const void* q,
                        const void* latent_kv, int32_t* out_idx, void* out, float* lse, void* ws, size_t ws_bytes,
                        dsa_stream_t stream) {
+  NvtxRange range("dsa_forward");
   dsa_status s = check_dims(dims, topk);
   if (s != DSA_OK) return s;
   const Layout L = make_layout(*dims, topk);

@@ -42,8 +42,12 @@ def test_workspace_bytes(dsa):
     prod = dsa.make_dims(1, 4096, 4096)
     n = dsa.dsa_workspace_bytes(prod, 2048)
     assert n >= 4096 * 2048 * 4 and n % 256 == 0
+    # decode rows up to 131072 keys keep every key's score (4 B); longer rows keep a top-k list
+    # of (key, position) pairs per 8192-key chunk
     dec = dsa.make_dims(64, 1, 131072)
-    assert dsa.dsa_workspace_bytes(dec, 2048) >= 64 * 16 * 2048 * 8
+    assert dsa.dsa_workspace_bytes(dec, 2048) >= 64 * 131072 * 4
+    long_rows = dsa.make_dims(4, 1, 140000)
+    assert dsa.dsa_workspace_bytes(long_rows, 2048) >= 4 * ((140000 + 8191) // 8192) * 2048 * 8
     tiny = dsa.make_dims(1, 512, 512, 4, 32, 8, 64, 16)
     assert dsa.dsa_workspace_bytes(tiny, 64) > dsa.dsa_workspace_bytes(dsa.make_dims(1, 512, 512), 64)  # padding
     for bad in [dsa.make_dims(1, 10, 5), dsa.make_dims(-1, 1, 1), dsa.make_dims(1, 1, 1, n_idx_heads=65),
