@@ -37,9 +37,9 @@ normalisation, KL), to scipy's softmax and relative entropy, to its closed forms
 (zero for scores = ln p + c, two points, one-hot) and to Gibbs' inequality, and
 its per-query term to padding and order invariance; the masked dense mode to
 torch's scaled_dot_product_attention in float64 with a boolean mask and to the
-sparse attention over the unmasked rows. Absolute values
-at the production shapes have no printed example on the pages: beyond these
-invariants and reductions they are parity-unpinned by the pages.
+sparse attention over the unmasked rows. The pages print no worked example,
+so no pin uses a printed value; every function here is pinned by the checks
+above, and the values at the production shapes rest on them.
 """
 from __future__ import annotations
 
